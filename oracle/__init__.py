@@ -1,0 +1,201 @@
+"""Plain fp64 CPU oracle for the Token Radius Attention hot path.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``; never by the product package.
+It shares no code with the CUDA path.  The arithmetic lives in
+``tra_oracle.c`` (compiled with gcc, fp64, OpenMP over queries); this module
+only compiles it and marshals numpy arrays.
+
+Every function works on the natural (frame-major) token order
+n = (t*H + h)*W + w of the "Token Radius Attention" blog post, sections 5.1
+and 9.1, with per-head arrays laid out [heads][N][...].
+
+Parity status of each function (what pins it) is listed in the repository's
+design notes; every function here is pinned by a CPU test.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tra_oracle.c")
+_OUT = os.path.join(_HERE, "_build", "libtra_oracle.so")
+_lib = None
+
+_I64P = ctypes.POINTER(ctypes.c_int64)
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_F32P = ctypes.POINTER(ctypes.c_float)
+_F64P = ctypes.POINTER(ctypes.c_double)
+_U8P = ctypes.POINTER(ctypes.c_uint8)
+
+
+def build(force: bool = False) -> str:
+    """Compile tra_oracle.c into oracle/_build/libtra_oracle.so."""
+    if not force and os.path.exists(_OUT) and os.path.getmtime(_OUT) >= os.path.getmtime(_SRC):
+        return _OUT
+    os.makedirs(os.path.dirname(_OUT), exist_ok=True)
+    tmp = _OUT + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+           "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _OUT)
+    return _OUT
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        L.oracle_decay_table.argtypes = [ctypes.c_double, ctypes.c_int, _F64P]
+        L.oracle_halfwidth.argtypes = [ctypes.c_int64, ctypes.c_double]
+        L.oracle_halfwidth.restype = ctypes.c_int64
+        L.oracle_rt_eff.argtypes = [ctypes.c_int, ctypes.c_int]
+        L.oracle_rt_eff.restype = ctypes.c_int
+        L.oracle_r_cap.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        L.oracle_r_cap.restype = ctypes.c_int64
+        L.oracle_count.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int] + [ctypes.c_int] * 3 + [ctypes.c_int64]
+        L.oracle_count.restype = ctypes.c_int64
+        L.oracle_budget.argtypes = [ctypes.c_float, ctypes.c_double, ctypes.c_double, ctypes.c_int64, ctypes.c_int64]
+        L.oracle_budget.restype = ctypes.c_int64
+        L.oracle_radius.argtypes = [_F32P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                    _I64P, ctypes.c_int64, _I32P, _I64P, _I64P]
+        L.oracle_token_mask.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int,
+                                                             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+        L.oracle_token_mask.restype = ctypes.c_int
+        L.oracle_block_mask.argtypes = [_I32P] + [ctypes.c_int] * 4 + [ctypes.c_double, ctypes.c_int] + \
+            [ctypes.c_int] * 4 + [_I64P, ctypes.c_int64, _U8P]
+        L.oracle_entropy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 5 + \
+            [ctypes.c_int] * 3 + [_I64P, ctypes.c_int64, _F64P]
+        L.oracle_attention.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, _I32P] + [ctypes.c_int] * 5 + \
+            [ctypes.c_double, ctypes.c_int, _I64P, ctypes.c_int64, _F64P]
+        L.oracle_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+def _elems(x: np.ndarray):
+    """(contiguous array, type flag) for the C side: 0 f32, 1 bf16 bits, 2 f64."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, 0
+    if x.dtype == np.uint16:
+        return x, 1
+    if x.dtype == np.float64:
+        return x, 2
+    raise TypeError(f"oracle takes float32, float64 or bf16 bits (uint16), got {x.dtype}")
+
+
+def _qlist(queries):
+    if queries is None:
+        return None, 0, None
+    q = np.ascontiguousarray(np.asarray(queries, dtype=np.int64))
+    return q, q.size, _ptr(q, _I64P)
+
+
+# ----------------------------------------------------------------- scalars
+def decay_table(gamma: float, rt_eff: int) -> np.ndarray:
+    g = np.zeros(rt_eff + 1, dtype=np.float64)
+    lib().oracle_decay_table(gamma, rt_eff, _ptr(g, _F64P))
+    return g
+
+
+def halfwidth(r: int, g: float) -> int:
+    return int(lib().oracle_halfwidth(r, g))
+
+
+def rt_eff(T: int, Rt: int) -> int:
+    return int(lib().oracle_rt_eff(T, Rt))
+
+
+def r_cap(T: int, H: int, W: int, gamma: float, Rt: int) -> int:
+    return int(lib().oracle_r_cap(T, H, W, gamma, Rt))
+
+
+def count(T, H, W, gamma, Rt, t, h, w, r) -> int:
+    return int(lib().oracle_count(T, H, W, gamma, Rt, t, h, w, r))
+
+
+def budget(Hent: float, a: float, b: float, N: int, Bmin: int) -> int:
+    return int(lib().oracle_budget(float(np.float32(Hent)), a, b, N, Bmin))
+
+
+def token_mask(T, H, W, gamma, Rt, i, j, r_i) -> bool:
+    return bool(lib().oracle_token_mask(T, H, W, gamma, Rt, i, j, r_i))
+
+
+# ----------------------------------------------------------------- arrays
+def radius(Hent, G, grid, a, b, gamma, Rt, Bmin, queries=None):
+    """E3+E4.  Hent: fp32 entropies (all G*N in order, or one per listed query).
+    Returns (r int32, c int64, bhat int64) per row."""
+    T, H, W = grid
+    Hf = np.ascontiguousarray(np.asarray(Hent, dtype=np.float32).reshape(-1))
+    q, nq, qp = _qlist(queries)
+    rows = nq if q is not None else G * T * H * W
+    assert Hf.size == rows
+    r = np.zeros(rows, np.int32)
+    c = np.zeros(rows, np.int64)
+    bh = np.zeros(rows, np.int64)
+    lib().oracle_radius(_ptr(Hf, _F32P), G, T, H, W, a, b, gamma, Rt, Bmin,
+                        qp, nq, _ptr(r, _I32P), _ptr(c, _I64P), _ptr(bh, _I64P))
+    return r, c, bh
+
+
+def block_mask(r, G, grid, gamma, Rt, qtile, ktile, qtiles=None) -> np.ndarray:
+    """E6.  r: int32 radii [G*N] natural order.  qtile/ktile: (th, tw) of the
+    (1, th, tw) query/key tiles.  Returns uint8 [rows, nK]: 0 inactive,
+    1 active, 3 active and full.  qtiles: list of g*nQ + a (None = all)."""
+    T, H, W = grid
+    rr = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
+    qth, qtw = qtile
+    kth, ktw = ktile
+    nQ = T * (-(-H // qth)) * (-(-W // qtw))
+    nK = T * (-(-H // kth)) * (-(-W // ktw))
+    q, nq, qp = _qlist(qtiles)
+    rows = nq if q is not None else G * nQ
+    out = np.zeros((rows, nK), np.uint8)
+    lib().oracle_block_mask(_ptr(rr, _I32P), G, T, H, W, gamma, Rt, qth, qtw, kth, ktw,
+                            qp, nq, _ptr(out, _U8P))
+    return out
+
+
+def entropy(q, k, G, grid, d, key_stride=1, ktile=(1, 1), queries=None) -> np.ndarray:
+    """E1 (key_stride 1) / E2 (key_stride > 1 over (1, kth, ktw) key tiles)."""
+    T, H, W = grid
+    qa, tq = _elems(q)
+    ka, tk = _elems(k)
+    assert tq == tk
+    ql, nq, qp = _qlist(queries)
+    rows = nq if ql is not None else G * T * H * W
+    out = np.zeros(rows, np.float64)
+    lib().oracle_entropy(qa.ctypes.data, ka.ctypes.data, tq, G, T, H, W, d,
+                         key_stride, ktile[0], ktile[1], qp, nq, _ptr(out, _F64P))
+    return out
+
+
+def attention(q, k, v, r, G, grid, d, gamma, Rt, queries=None) -> np.ndarray:
+    """E7: masked softmax attention, fp64 [rows, d]."""
+    T, H, W = grid
+    qa, tq = _elems(q)
+    ka, tk = _elems(k)
+    va, tv = _elems(v)
+    assert tq == tk == tv
+    rr = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
+    ql, nq, qp = _qlist(queries)
+    rows = nq if ql is not None else G * T * H * W
+    out = np.zeros((rows, d), np.float64)
+    lib().oracle_attention(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, tq, _ptr(rr, _I32P),
+                           G, T, H, W, d, gamma, Rt, qp, nq, _ptr(out, _F64P))
+    return out
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
