@@ -1,0 +1,455 @@
+"""Benchmark of the Token Radius Attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan720] [--impl tra|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+dense (or key-subsampled) warm-up entropy, one radius/mask build, then
+`calls` attention calls that reuse the mask with a fresh V each (10 for the
+Wan-14B-720p shape: 21x45x80 tokens, 40 heads, d=128, bf16).  The headline
+value is the retained-pair throughput of the attention calls: 4*d FLOPs per
+retained token pair (the pairs the radius mask keeps, not the padded tiles
+the kernel computes) over their device time, summed over ranks (heads are
+independent, so ranks run independent replicas: weak scaling, no collective
+on the data path).  Inputs are resident in HBM and larger than L2; L2 is
+also flushed before every step.
+
+`--impl reference` runs the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "TRA attention retained-pair TFLOP/s (bf16) at 21x45x80 tokens, 40 heads; ms/call reported"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def aggregate(per_rank_units: float, per_rank_seconds: float, world: int) -> float:
+    """Whole-job throughput: units of all ranks over the slowest rank's time."""
+    return per_rank_units * world / max_over_ranks(per_rank_seconds, world)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"tra_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- profiles
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    from sparse_attention_video_tra_b200.build import CSRC
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        h.update(open(os.path.join(CSRC, f), "rb").read())
+    if kv.get("source_sha256") != h.hexdigest():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+def oracle_sample(wl, b, budget_s: float, rng_seed: int, heads=(0,), device="cuda"):
+    """Time the fp64 oracle's whole path (entropy, radius, attention) on a
+    bounded random sample of queries of the same workload.  Returns the
+    retained-pair TFLOP/s it reached and a description."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    from sparse_attention_video_tra_b200 import synth
+    T, H, W, d = wl.T, wl.H, wl.W, wl.d
+    N = wl.N
+    q, k, v = synth.make_qkv(T, H, W, wl.heads, d, synth.SEED_BASE + wl.index, device=device,
+                             dtype=torch.bfloat16)
+    sel = list(heads)
+
+    def bits(x):
+        return x[sel].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    del q, k, v
+    G = len(sel)
+    rng = np.random.default_rng(rng_seed)
+    threads = oracle.num_threads()
+
+    def run(nq):
+        idx = np.sort(rng.choice(G * N, size=nq, replace=False))
+        t0 = time.perf_counter()
+        Hs = oracle.entropy(qb, kb, G, (T, H, W), d, key_stride=wl.key_stride, ktile=(8, 16), queries=idx) \
+            if wl.key_stride == 1 else _oracle_entropy_tiled(oracle, qb, kb, G, wl, idx)
+        r, c, _ = oracle.radius(Hs.astype(np.float32), G, (T, H, W), wl.a, b, wl.gamma, wl.Rt, wl.Bmin, queries=idx)
+        r_all = np.zeros(G * N, np.int32)
+        r_all[idx] = r
+        oracle.attention(qb, kb, vb, r_all, G, (T, H, W), d, wl.gamma, wl.Rt, queries=idx)
+        dt = time.perf_counter() - t0
+        return dt, int(c.sum()), nq
+
+    dt, pairs, nq = run(max(threads, 4))
+    if dt < budget_s / 4:
+        n2 = int(min(G * N, max(nq, nq * budget_s / max(dt, 1e-3))))
+        dt, pairs, nq = run(n2)
+    tflops = 4.0 * d * pairs / dt / 1e12
+    return tflops, {"queries": nq, "heads": sel, "seconds": round(dt, 3), "threads": threads,
+                    "retained_pairs": pairs}
+
+
+def _oracle_entropy_tiled(oracle, qb, kb, G, wl, idx):
+    # key subsampling is defined on the library's key tiles: pass the plan's tile shape
+    from sparse_attention_video_tra_b200 import Plan
+    p = Plan(wl.T, wl.H, wl.W, 1, wl.d, 1.0, 0.0, wl.gamma, wl.Rt, wl.Bmin)
+    th, tw = p.info.tile_h, p.info.tile_w
+    p.close()
+    return oracle.entropy(qb, kb, G, (wl.T, wl.H, wl.W), wl.d, key_stride=wl.key_stride, ktile=(th, tw), queries=idx)
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    sys.path.insert(0, ROOT)
+    from sparse_attention_video_tra_b200 import synth
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    # b for the target retained fraction, found with the oracle on a query sample
+    b = wl.b
+    if b is None:
+        b = _oracle_calibrate_b(oracle, wl, dev)
+    vals = []
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for s in range(args.warmup + args.steps):
+        v, desc = oracle_sample(wl, b, budget, 1234 + s, device=dev)
+        if s >= args.warmup:
+            vals.append((v, desc))
+    value = float(np.mean([v for v, _ in vals]))
+    desc = vals[-1][1]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "b": b, "sample": "random queries of head 0, whole oracle path"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": desc["threads"], "kind": "oracle",
+                             "sample": f"{desc['queries']} queries of head 0 per step, entropy+radius+attention"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _oracle_calibrate_b(oracle, wl, dev):
+    from sparse_attention_video_tra_b200 import synth
+    q, k, _ = synth.make_qkv(wl.T, wl.H, wl.W, wl.heads, wl.d, synth.SEED_BASE + wl.index, device=dev,
+                             dtype=torch.bfloat16)
+    qb = q[:1].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    kb = k[:1].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    del q, k
+    rng = np.random.default_rng(99)
+    idx = np.sort(rng.choice(wl.N, size=256, replace=False))
+    if wl.key_stride == 1:
+        Hs = oracle.entropy(qb, kb, 1, wl.grid, wl.d, queries=idx)
+    else:
+        Hs = _oracle_entropy_tiled(oracle, qb, kb, 1, wl, idx)
+    lo, hi = -30.0, 30.0
+    for _ in range(30):
+        mid = 0.5 * (lo + hi)
+        _, c, _ = oracle.radius(Hs.astype(np.float32), 1, wl.grid, wl.a, mid, wl.gamma, wl.Rt, wl.Bmin, queries=idx)
+        if c.mean() / wl.N < wl.target_retained:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+def run_tra(args, rank, world):
+    sys.path.insert(0, ROOT)
+    from sparse_attention_video_tra_b200 import Plan, synth
+    from sparse_attention_video_tra_b200.runner import WorkloadRun
+    wl = synth.WORKLOADS[args.workload]
+    calls = args.calls if args.calls else (10 if args.workload == "wan720" else 1)
+    run = WorkloadRun(wl, calls=calls, seed_offset=rank)
+    dev_idx = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    nev = 3 + calls
+
+    def timed_steps(k, record):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(k)]
+        for s in range(k):
+            flush.zero_()
+            run.step(evs[s] if record else None, stream=None)
+        return evs
+
+    for _ in range(args.warmup):
+        timed_steps(1, False)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = ClockSampler(dev_idx)
+    clocks.start()
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall0 = time.perf_counter()
+    evs = timed_steps(args.steps, True)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    barrier(world)
+    clk = clocks.stop()
+
+    step_ms = [e[0].elapsed_time(e[-1]) for e in evs]
+    ent_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    mask_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    call_ms = [e[2 + c].elapsed_time(e[3 + c]) for e in evs for c in range(calls)]
+    attn_s = sum(call_ms) / 1000.0
+    flops = run.attention_flops()
+    value = aggregate(flops * calls * args.steps, attn_s, world) / 1e12
+    step_s = sum(step_ms) / 1000.0
+    step_tflops = aggregate(flops * calls * args.steps, step_s, world) / 1e12
+    ms_per_step = max_over_ranks(float(np.mean(step_ms)), world)
+
+    # separate L2-flushed timing of the mask build (its inputs fit in L2)
+    mask_runs = []
+    for _ in range(5):
+        flush.zero_()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        run.run_mask()
+        a1.record()
+        torch.cuda.synchronize()
+        mask_runs.append(a0.elapsed_time(a1))
+    mask_cold_ms = float(np.median(mask_runs))
+
+    pk, pk_kind = peaks()
+    avg_call_s = attn_s / (calls * args.steps)
+    achieved = flops / avg_call_s / 1e12
+    peak = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    computed = run.computed_pairs()
+    traffic = recorded_traffic("attention", args.workload)
+    roofline = {"bound": "tensor", "kernel": "tra::attention_kernel", "achieved": round(achieved, 2),
+                "peak": peak, "peak_kind": f"{pk_kind} bf16 sustained", "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "computed_tile_tflops": round(4.0 * wl.d * computed / avg_call_s / 1e12, 2),
+                "computed_tile_frac": round(4.0 * wl.d * computed / avg_call_s / 1e12 / peak, 4),
+                "tile_efficiency": round(run.retained_pairs / computed, 4),
+                "frac_of_burst": round(achieved / float(pk.get("bf16_tflops", 1590.0)), 4)}
+    mask_bytes_alg = mask_algorithmic_bytes(run)
+    phases = {"entropy_ms": round(float(np.mean(ent_ms)), 3), "mask_ms": round(float(np.mean(mask_ms)), 4),
+              "mask_ms_l2_flushed": round(mask_cold_ms, 4),
+              "mask_hbm_frac": round(mask_bytes_alg / (mask_cold_ms / 1000.0) / 1e9 / float(pk.get("hbm_gbs", 6650.0)), 4),
+              "attention_ms_per_call": round(float(np.mean(call_ms)), 3),
+              "entropy_scores_per_s": run.entropy_pairs() / (float(np.mean(ent_ms)) / 1000.0)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, desc = oracle_sample(wl, run.b, args.cpu_budget, 4321)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": desc["threads"], "kind": "oracle",
+               "sample": f"{desc['queries']} random queries of head 0: entropy+radius+attention in fp64, "
+                         f"{desc['seconds']} s"}
+
+    e2e = None if args.no_e2e else run_e2e(run, wl, calls, args, world)
+    b_used, retained = run.b, run.retained_fraction_now()
+    del run
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Q,K,V with Wan-720p attention shapes; no model weights)",
+            "config": {"workload": wl.name, "global_batch": wl.heads * world, "seq_len": wl.N,
+                       "parallelism": f"independent head-batch replicas x{world}", "attention_calls_per_step": calls,
+                       "a": wl.a, "b": round(b_used, 6), "gamma": wl.gamma, "Rt": wl.Rt, "Bmin": wl.Bmin,
+                       "inputs": "resident in HBM, 774 MB per tensor (> L2); L2 flushed before every step"},
+            "retained_fraction": round(retained, 5), "phases": phases, "step_tflops": round(step_tflops, 3),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": (2 + calls) * args.steps, "clocks": clk, "wall_s_timed": round(t_wall, 3)}
+    return line
+
+
+def mask_algorithmic_bytes(run) -> float:
+    """Bytes the mask build must move: read H (4 B/row), write r (4 B/row),
+    per tile count (4 B) and pair sum (8 B), 2 B per listed key tile."""
+    i = run.info
+    listed = int(run.plan.mask_views(run.mask)[1].sum().item())
+    return i.heads * i.N_pad * 8.0 + i.heads * i.n_tiles * 12.0 + 2.0 * listed
+
+
+def run_e2e(run, wl, calls, args, world):
+    """The same metric through the public API with host buffers: per step,
+    pinned host -> device copies of Q, K and each call's V (natural order),
+    tile-major permutes, the hot path, and each call's output back to host."""
+    from sparse_attention_video_tra_b200 import Plan
+    i = run.info
+    plan = run.plan
+    shape = (i.heads, i.N, i.d)
+    hq = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    hk = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    hv = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    ho = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    tmp = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    plan.permute(run.q, tmp, False); hq.copy_(tmp)
+    plan.permute(run.k, tmp, False); hk.copy_(tmp)
+    plan.permute(run.v[0], tmp, False); hv.copy_(tmp)
+    dq, dk, dv, dn = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    del tmp
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        plan.permute(dq, run.q)
+        plan.permute(dk, run.k)
+        plan.entropy(run.q, run.k, run.H, wl.key_stride)
+        plan.radius_and_mask(run.H, run.mask)
+        for c in range(calls):
+            dv.copy_(hv, non_blocking=True)
+            plan.permute(dv, run.v[c])
+            plan.attention(run.q, run.k, run.v[c], run.mask, run.out)
+            plan.permute(run.out, dn, False)
+            ho.copy_(dn, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    secs = e0.elapsed_time(e1) / 1000.0
+    val = aggregate(run.attention_flops() * calls * args.steps, secs, world) / 1e12
+    nbytes = i.heads * i.N * i.d * 2
+    return {"value": round(val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": nbytes * (2 + calls),
+            "d2h_bytes_per_step": nbytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3)}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="tra", choices=["tra", "reference"])
+    ap.add_argument("--workload", default="wan720")
+    ap.add_argument("--calls", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    rank, world = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        line = run_tra(args, rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

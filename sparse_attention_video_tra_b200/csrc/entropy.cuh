@@ -1,0 +1,194 @@
+// entropy.cuh -- per-query softmax entropy of the warm-up attention, on the
+// sm_100a tensor cores (tcgen05 + TMEM), K tiles staged by TMA.
+//
+// "Token Radius Attention for Efficient Video Generation" (gist.science
+// summary), section 2, "Entropie-vers-Budget": a dense warm-up step measures
+// every query's attention entropy, which later steps reuse; the daily-ai-
+// frontier TL;DR of the same paper calls it fused entropy extraction.
+//
+// With u_j = (q.k_j / sqrt d) * log2(e) and a running maximum m, the kernel
+// keeps Z = sum_j 2^(u_j - m) and A = sum_j 2^(u_j - m) (u_j - m); then
+//   H = -sum_j p_j ln p_j = ln Z - ln(2) * A / Z.
+// When m grows to m': A <- 2^(m-m') (A + (m - m') Z), Z <- 2^(m-m') Z.
+// Key subsampling (key_tile_stride s > 1) visits the key tiles whose index is
+// a multiple of s and adds ln(N / |S|) (host-computed) so that a uniform
+// distribution still reads ln N.
+//
+// One CTA per (query tile of 128 tokens, head), two CTAs per SM.  192 threads:
+//   warps 0-3 statistics (thread i = query row i = TMEM lane i),
+//   warp 4 TMA producer (Q, then the K ring), warp 5 TMEM allocator + MMA
+//   issuer (S[j%2] = Q K_j^T, two 128-column fp32 buffers).
+#pragma once
+#include "pipeline.cuh"
+
+namespace tra {
+
+template <int D>
+struct EntCfg {
+    static constexpr int PANEL = 128 * 128;
+    static constexpr int NP = D / 64;
+    static constexpr int TILE = NP * PANEL;
+    static constexpr int KST = (D == 128) ? 2 : 3;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = TILE;
+    static constexpr int OFF_BAR = OFF_K + KST * TILE;
+    static constexpr int NBAR = 1 + 2 * KST + 4 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static constexpr int THREADS = 192;
+};
+
+template <int D, int TWL>
+__global__ void __launch_bounds__(192, 2)
+entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const Geom G, int stride, float corr, float* __restrict__ Hout)
+{
+    using C = EntCfg<D>;
+    constexpr int TW = 1 << TWL;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem + C::OFF_Q;
+    uint8_t* sK = smem + C::OFF_K;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = k_full + C::KST;
+    uint64_t* s_full = k_empty + C::KST;
+    uint64_t* s_empty = s_full + 2;
+    uint64_t* drain = s_empty + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    const int tile = blockIdx.x, g = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = (G.nQ + stride - 1) / stride;              // key tiles visited
+    const int row0 = g * G.N_pad + tile * 128;
+
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < C::KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 128); }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) { tmem_alloc(s_tmem, 256); tmem_relinquish(); }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_q); prefetch_tmap(&tm_k);
+            mbar_arrive_expect_tx(q_full, C::TILE);
+#pragma unroll
+            for (int p = 0; p < C::NP; ++p) tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, row0, q_full);
+            int issued = 0;
+            for (int j = 0; j < n; ++j) {
+                const int st = j % C::KST;
+                if (j >= C::KST && !role_wait(&k_empty[st], ((j / C::KST) - 1) & 1, G.wait_ns, s_abort)) break;
+                mbar_arrive_expect_tx(&k_full[st], C::TILE);
+#pragma unroll
+                for (int p = 0; p < C::NP; ++p)
+                    tma_load_2d(sK + st * C::TILE + p * C::PANEL, &tm_k, p * 64, g * G.N_pad + j * stride * 128,
+                                &k_full[st]);
+                ++issued;
+            }
+            mbar_wait(q_full, 0, G.drain_ns);
+            for (int j = max(0, issued - C::KST); j < issued; ++j)
+                mbar_wait(&k_full[j % C::KST], (j / C::KST) & 1, G.drain_ns);
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false);
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+            bool ok = role_wait(q_full, 0, G.wait_ns, s_abort);
+            for (int j = 0; ok && j < n; ++j) {
+                const int ks = j % C::KST;
+                if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) break;
+                if (j >= 2 && !role_wait(&s_empty[j & 1], ((j - 2) >> 1) & 1, G.wait_ns, s_abort)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
+                    mma_ss(tmem + (j & 1) * 128, smem_desc_sw128(sQa + off, 16, 1024),
+                           smem_desc_sw128(sKa + ks * C::TILE + off, 16, 1024), IDESC, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[j & 1]);
+                mma_commit(&k_empty[ks]);
+            }
+            mma_commit(drain);
+            mbar_wait(drain, 0, G.drain_ns);
+        }
+    } else {
+        const int row = tid;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float c = G.scale_log2;
+        float m = -1e30f, Z = 0.f, A = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const int kb = j * stride;
+            int tk, trk, tck;
+            tile_coords(G, kb, tk, trk, tck);
+            const int khv = min(G.th, G.H - trk * G.th), kwv = min(TW, G.W - tck * TW);
+            const bool edge = khv < G.th || kwv < TW;
+            const int bs = j & 1;
+            const bool got = role_wait(&s_full[bs], (j >> 1) & 1, G.wait_ns, s_abort);
+            if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
+            tc_fence_after();
+            __syncwarp();
+            float s[128];
+            {
+                uint32_t v[32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    tmem_ld32(tmem + lane_base + bs * 128 + q * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(v[i]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&s_empty[bs]);
+            if (edge) {                     // pad keys of edge tiles take no probability
+                uint32_t keep[4];
+                row_keep_bits<TWL>(0, khv - 1, 0, kwv - 1, keep);
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                    if (!((keep[i >> 5] >> (i & 31)) & 1u)) s[i] = -1e30f;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+            const float mt = mx * c;
+            if (mt > m) {
+                const float alpha = ex2(m - mt);
+                A = alpha * fmaf(m - mt, Z, A);
+                Z *= alpha;
+                m = mt;
+            }
+            float zt = 0.f, at = 0.f;
+#pragma unroll
+            for (int i = 0; i < 128; ++i) {
+                const float u = fmaf(s[i], c, -m);
+                const float e = ex2(u);
+                zt += e;
+                at = fmaf(e, u, at);
+            }
+            Z += zt;
+            A += at;
+        }
+        if (ok) {
+            const float H = logf(Z) - 0.69314718055994531f * (A / Z) + corr;
+            Hout[row0 + row] = H;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace tra

@@ -1,0 +1,180 @@
+// radius_mask.cuh -- budget, radius and block-sparse mask in one launch.
+//
+// "Token Radius Attention for Efficient Video Generation" (gist.science
+// summary), section 2: Intuition I (entropy -> token budget), "Budget-vers-
+// Rayon" (budget -> query radius, shrunk per frame by the temporal decay), and
+// "Noyaux CUDA Fusionnes" (distance computation, radius comparison, block
+// pruning and token voting fused into one kernel that emits a block-sparse
+// mask).  Token voting is read as an OR vote: a key tile is listed for a query
+// tile iff some retained token pair falls in it, so skipping unlisted tiles
+// never changes the attention output.
+//
+// One CTA per (query tile, head), one thread per tile row (token).
+//   1. Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))) in fp64.
+//   2. r = the smallest r in [0, r_cap] whose clipped neighbourhood count
+//      reaches Bhat (binary search; the count is monotone in r).
+//   3. Per frame distance |dt|: every query's neighbourhood is a rectangle of
+//      key tiles that contains the query tile's own tile position, so for a
+//      key tile row the union over the tile's queries is one interval of tile
+//      columns (warp min/max reductions), and the "full" tiles (every valid
+//      pair retained) are the intersection of per-query rectangles.
+//   4. The active tiles of the frames within Rt' are written in ascending
+//      tile order after a block-wide prefix sum over (frame, tile row).
+#pragma once
+#include "tra_common.cuh"
+
+namespace tra {
+
+// clipped neighbourhood count c(r) of the query at (t, h, w)
+__device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int w, int r)
+{
+    long long c = 0;
+    for (int dl = 0; dl <= G.rte; ++dl) {
+        const int m = (t + dl < G.T ? 1 : 0) + (dl > 0 && t - dl >= 0 ? 1 : 0);
+        if (m == 0) break;                         // farther frames are out of the grid too
+        const int s = halfwidth(r, G.g[dl]);
+        const int X = min(h, s) + min(G.H - 1 - h, s) + 1;
+        const int Y = min(w, s) + min(G.W - 1 - w, s) + 1;
+        c += (long long)(m * X) * Y;
+    }
+    return c;
+}
+
+__device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
+{
+    const double x = __dadd_rn(__dmul_rn(G.a, (double)Hent), G.b);
+    const double e = exp(x);
+    const double B = fmin((double)G.N, fmax((double)G.Bmin, e));
+    return (long long)ceil(B);
+}
+
+__global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
+                                                          uint8_t* __restrict__ mask)
+{
+    __shared__ int s_lo[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];
+    __shared__ int s_hi[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];
+    __shared__ int s_full[TRA_MAX_RT_EFF + 1][4];
+    __shared__ int s_len[TRA_MAX_LIST_ROWS];
+    __shared__ long long s_pairs[4];
+    __shared__ int s_warp[4];
+
+    const int tile = blockIdx.x, g = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int t, trq, tcq;
+    tile_coords(G, tile, t, trq, tcq);
+    const int h = trq * G.th + (tid >> G.tw_log2);
+    const int w = tcq * G.tw + (tid & (G.tw - 1));
+    const bool valid = h < G.H && w < G.W;
+    const size_t row = (size_t)g * G.N_pad + (size_t)tile * 128 + tid;
+
+    for (int i = tid; i < (G.rte + 1) * TRA_MAX_TILES_H; i += 128) {
+        (&s_lo[0][0])[i] = 0x7fffffff;
+        (&s_hi[0][0])[i] = -1;
+    }
+    if (tid < G.rte + 1) {
+        s_full[tid][0] = -0x7fffffff; s_full[tid][1] = 0x7fffffff;
+        s_full[tid][2] = -0x7fffffff; s_full[tid][3] = 0x7fffffff;
+    }
+
+    // ---- budget and radius
+    int r = -1;
+    long long c = 0;
+    if (valid) {
+        const long long bh = budget_hat(G, Hent[row]);
+        int lo = 0, hi = G.r_cap;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (nbr_count(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+        }
+        r = lo;
+        c = nbr_count(G, t, h, w, r);
+    }
+    reinterpret_cast<int32_t*>(mask + G.off_radius)[row] = r;
+
+    // ---- retained pairs of the tile
+    long long cs = c;
+    for (int o = 16; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
+    if (lane == 0) s_pairs[warp] = cs;
+    __syncthreads();
+    if (tid == 0)
+        reinterpret_cast<long long*>(mask + G.off_pairs)[(size_t)g * G.nQ + tile] =
+            s_pairs[0] + s_pairs[1] + s_pairs[2] + s_pairs[3];
+
+    // ---- per frame distance: active tile-column interval per tile row, full rectangle
+    for (int dl = 0; dl <= G.rte; ++dl) {
+        if (!(t + dl < G.T || t - dl >= 0)) break;    // uniform over the CTA
+        int rl = 0x7fffffff, rh = -1, cl = 0, ch = -1;
+        int frl = -0x7fffffff, frh = 0x7fffffff, fcl = -0x7fffffff, fch = 0x7fffffff;
+        if (valid) {
+            const int s = halfwidth(r, G.g[dl]);
+            rl = max(0, h - s) >> G.th_log2;
+            rh = min(G.H - 1, h + s) >> G.th_log2;
+            cl = max(0, w - s) >> G.tw_log2;
+            ch = min(G.W - 1, w + s) >> G.tw_log2;
+            frl = (h - s <= 0) ? 0 : ((h - s + G.th - 1) >> G.th_log2);
+            frh = (h + s >= G.H - 1) ? G.nTh - 1 : (((h + s + 1) >> G.th_log2) - 1);
+            fcl = (w - s <= 0) ? 0 : ((w - s + G.tw - 1) >> G.tw_log2);
+            fch = (w + s >= G.W - 1) ? G.nTw - 1 : (((w + s + 1) >> G.tw_log2) - 1);
+        }
+        frl = __reduce_max_sync(0xffffffffu, frl);
+        frh = __reduce_min_sync(0xffffffffu, frh);
+        fcl = __reduce_max_sync(0xffffffffu, fcl);
+        fch = __reduce_min_sync(0xffffffffu, fch);
+        if (lane == 0) {
+            atomicMax(&s_full[dl][0], frl); atomicMin(&s_full[dl][1], frh);
+            atomicMax(&s_full[dl][2], fcl); atomicMin(&s_full[dl][3], fch);
+        }
+        const int r_lo = __reduce_min_sync(0xffffffffu, rl);
+        const int r_hi = __reduce_max_sync(0xffffffffu, rh);
+        for (int tr = r_lo; tr <= r_hi; ++tr) {
+            const bool in = rl <= tr && tr <= rh;
+            const int lo = __reduce_min_sync(0xffffffffu, in ? cl : 0x7fffffff);
+            const int hi = __reduce_max_sync(0xffffffffu, in ? ch : -1);
+            if (lane == 0 && hi >= 0) {
+                atomicMin(&s_lo[dl][tr], lo);
+                atomicMax(&s_hi[dl][tr], hi);
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- list rows (frame, tile row) in ascending tile order; block prefix sum
+    const int t0 = max(0, t - G.rte), t1 = min(G.T - 1, t + G.rte);
+    const int R = (t1 - t0 + 1) * G.nTh;
+    for (int i = tid; i < R; i += 128) {
+        const int f = i / G.nTh, tr = i - f * G.nTh;
+        const int dl = abs(t0 + f - t);
+        s_len[i] = s_hi[dl][tr] >= 0 ? s_hi[dl][tr] - s_lo[dl][tr] + 1 : 0;
+    }
+    __syncthreads();
+    const int per = (R + 127) >> 7;
+    const int beg = min(R, tid * per), end = min(R, beg + per);
+    int local = 0;
+    for (int i = beg; i < end; ++i) local += s_len[i];
+    int incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int off = incl - local;
+    for (int k = 0; k < warp; ++k) off += s_warp[k];
+    uint16_t* list = reinterpret_cast<uint16_t*>(mask + G.off_list) + ((size_t)g * G.nQ + tile) * G.list_cap;
+    for (int i = beg; i < end; ++i) {
+        const int f = i / G.nTh, tr = i - f * G.nTh;
+        const int dl = abs(t0 + f - t);
+        const int lo = s_lo[dl][tr], hi = s_hi[dl][tr];
+        const bool row_full = s_full[dl][0] <= tr && tr <= s_full[dl][1];
+        const int base = ((t0 + f) * G.nTh + tr) * G.nTw;
+        for (int tc = lo; tc <= hi; ++tc) {
+            const bool full = row_full && s_full[dl][2] <= tc && tc <= s_full[dl][3];
+            list[off++] = (uint16_t)((base + tc) | (full ? 0x8000 : 0));
+        }
+    }
+    if (tid == 0)
+        reinterpret_cast<int32_t*>(mask + G.off_count)[(size_t)g * G.nQ + tile] =
+            s_warp[0] + s_warp[1] + s_warp[2] + s_warp[3];
+}
+
+}  // namespace tra

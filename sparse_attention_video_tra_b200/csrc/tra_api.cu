@@ -1,0 +1,188 @@
+// tra_api.cu -- the extern "C" entry points that launch the kernels: argument
+// checks, TMA tensor maps, kernel selection by (head dim, tile width), and the
+// device error word.  All kernels are compiled into this one translation unit.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/tra.h"
+#include "tra_plan_impl.h"
+#include "pipeline.cuh"
+#include "permute.cuh"
+#include "radius_mask.cuh"
+#include "entropy.cuh"
+#include "attention.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [rows][D] bf16 rows, 128-row x 64-column boxes, 128-byte swizzle
+bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, int D)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+tra_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? TRA_OK : TRA_ERR_CUDA;
+}
+
+template <class K>
+bool set_smem(K kernel, int bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+template <int D, int TWL>
+tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                         const uint8_t* mask, __nv_bfloat16* out, cudaStream_t st)
+{
+    using C = tra::AttnCfg<D>;
+    auto kern = tra::attention_kernel<D, TWL>;
+    if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
+    kern<<<dim3(G.nQ, G.G), C::THREADS, C::SMEM, st>>>(q, k, v, G, mask, out);
+    return launch_status();
+}
+
+template <int D, int TWL>
+tra_status run_entropy(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, int stride, float corr,
+                       float* H, cudaStream_t st)
+{
+    using C = tra::EntCfg<D>;
+    auto kern = tra::entropy_kernel<D, TWL>;
+    if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
+    kern<<<dim3(G.nQ, G.G), C::THREADS, C::SMEM, st>>>(q, k, G, stride, corr, H);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" tra_status tra_permute(tra_plan plan, const void* src, void* dst, int to_tile_major, tra_stream stream)
+{
+    if (!plan || !src || !dst || !aligned(src, 16) || !aligned(dst, 16)) return TRA_ERR_INVALID_ARG;
+    const tra::Geom& G = plan->geom;
+    const size_t total = (size_t)G.G * G.N_pad * (G.D / 8);
+    const int blocks = (int)std::min<size_t>((total + 255) / 256, 148 * 32);
+    tra::permute_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(G, (const uint4*)src, (uint4*)dst,
+                                                                   to_tile_major ? 1 : 0);
+    return launch_status();
+}
+
+extern "C" tra_status tra_entropy(tra_plan plan, const void* q, const void* k, float* Hout, int key_tile_stride,
+                                  tra_stream stream)
+{
+    if (!plan || !q || !k || !Hout || !aligned(q, 16) || !aligned(k, 16) || !aligned(Hout, 4))
+        return TRA_ERR_INVALID_ARG;
+    const tra::Geom& G = plan->geom;
+    if (key_tile_stride < 1 || key_tile_stride > G.nQ) return TRA_ERR_INVALID_ARG;
+    // |S| = valid keys in the sampled tiles; corr = ln(N / |S|)
+    float corr = 0.f;
+    if (key_tile_stride > 1) {
+        long long nS = 0;
+        for (int kb = 0; kb < G.nQ; kb += key_tile_stride) {
+            const int rem = kb % G.tiles_per_frame;
+            const int tr = rem / G.nTw, tc = rem % G.nTw;
+            nS += (long long)std::min(G.th, G.H - tr * G.th) * std::min(G.tw, G.W - tc * G.tw);
+        }
+        corr = (float)std::log((double)G.N / (double)nS);
+    }
+    CUtensorMap mq, mk;
+    const uint64_t rows = (uint64_t)G.G * G.N_pad;
+    if (!make_row_map(&mq, q, rows, G.D) || !make_row_map(&mk, k, rows, G.D)) return TRA_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int key = G.D * 100 + G.tw_log2;
+    switch (key) {
+        case 6402: return run_entropy<64, 2>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 6403: return run_entropy<64, 3>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 6404: return run_entropy<64, 4>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 6405: return run_entropy<64, 5>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 12802: return run_entropy<128, 2>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 12803: return run_entropy<128, 3>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 12804: return run_entropy<128, 4>(G, mq, mk, key_tile_stride, corr, Hout, st);
+        case 12805: return run_entropy<128, 5>(G, mq, mk, key_tile_stride, corr, Hout, st);
+    }
+    return TRA_ERR_UNSUPPORTED;
+}
+
+extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void* mask, size_t mask_bytes,
+                                          tra_stream stream)
+{
+    if (!plan || !Hent || !mask || !aligned(Hent, 4) || !aligned(mask, 256)) return TRA_ERR_INVALID_ARG;
+    if (mask_bytes < plan->mask_bytes) return TRA_ERR_WORKSPACE;
+    const tra::Geom& G = plan->geom;
+    tra::radius_mask_kernel<<<dim3(G.nQ, G.G), 128, 0, (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
+    return launch_status();
+}
+
+extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k, const void* v, const void* mask,
+                                    void* out, tra_stream stream)
+{
+    if (!plan || !q || !k || !v || !mask || !out) return TRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(mask, 256))
+        return TRA_ERR_INVALID_ARG;
+    const tra::Geom& G = plan->geom;
+    CUtensorMap mq, mk, mv;
+    const uint64_t rows = (uint64_t)G.G * G.N_pad;
+    if (!make_row_map(&mq, q, rows, G.D) || !make_row_map(&mk, k, rows, G.D) || !make_row_map(&mv, v, rows, G.D))
+        return TRA_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    const uint8_t* m = (const uint8_t*)mask;
+    __nv_bfloat16* o = (__nv_bfloat16*)out;
+    const int key = G.D * 100 + G.tw_log2;
+    switch (key) {
+        case 6402: return run_attention<64, 2>(G, mq, mk, mv, m, o, st);
+        case 6403: return run_attention<64, 3>(G, mq, mk, mv, m, o, st);
+        case 6404: return run_attention<64, 4>(G, mq, mk, mv, m, o, st);
+        case 6405: return run_attention<64, 5>(G, mq, mk, mv, m, o, st);
+        case 12802: return run_attention<128, 2>(G, mq, mk, mv, m, o, st);
+        case 12803: return run_attention<128, 3>(G, mq, mk, mv, m, o, st);
+        case 12804: return run_attention<128, 4>(G, mq, mk, mv, m, o, st);
+        case 12805: return run_attention<128, 5>(G, mq, mk, mv, m, o, st);
+    }
+    return TRA_ERR_UNSUPPORTED;
+}
+
+extern "C" tra_status tra_plan_status(tra_plan plan)
+{
+    (void)plan;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, tra::g_tra_error, sizeof word) != cudaSuccess) return TRA_ERR_CUDA;
+    if (word) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(tra::g_tra_error, &zero, sizeof zero) != cudaSuccess) return TRA_ERR_CUDA;
+    }
+    if (word & TRA_ERRBIT_TIMEOUT) return TRA_ERR_TIMEOUT;
+    if (word & TRA_ERRBIT_CHECK) return TRA_ERR_DEVICE_CHECK;
+    return TRA_OK;
+}

@@ -1,0 +1,31 @@
+// tra_geom.h -- the plan as seen by the kernels: plain data, passed by value
+// to every launch.  Built on the host by the plan code (tra_plan.cpp).
+#pragma once
+#include <cstdint>
+
+#define TRA_MAX_RT_EFF 31            // decay table holds gamma^0 .. gamma^31
+#define TRA_MAX_TILES_H 64           // tile rows per frame the mask kernel handles
+#define TRA_MAX_LIST_ROWS 4096       // (2Rt'+1) * tile rows per frame
+#define TRA_MAX_R_CAP (1 << 20)
+#define TRA_MAX_LIST_CAP 4096         // key tiles listed per query tile
+#define TRA_ERRBIT_TIMEOUT 1u
+#define TRA_ERRBIT_CHECK 2u
+
+namespace tra {
+
+struct Geom {
+    int T, H, W, G, D;               // grid, heads, head dim
+    int N, N_pad;                    // tokens per head, tile-major rows per head
+    int th, tw, th_log2, tw_log2;    // (1, th, tw) tiles, th*tw = 128
+    int nTh, nTw, tiles_per_frame, nQ;
+    int rte, r_cap, list_cap;
+    int Bmin;
+    double a, b;
+    double g[TRA_MAX_RT_EFF + 1];    // gamma^delta
+    long long off_radius, off_count, off_pairs, off_list;
+    float scale_log2;                // log2(e) / sqrt(d)
+    unsigned long long wait_ns;      // limit of a pipeline wait
+    unsigned long long drain_ns;     // limit of the waits that drain in-flight copies
+};
+
+}  // namespace tra
