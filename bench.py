@@ -189,10 +189,11 @@ def oracle_sample(wl, b, budget_s: float, rng_seed: int, heads=(0,), device="cud
         dt = time.perf_counter() - t0
         return dt, int(c.sum()), nq
 
-    dt, pairs, nq = run(max(threads, 4))
-    if dt < budget_s / 4:
-        n2 = int(min(G * N, max(nq, nq * budget_s / max(dt, 1e-3))))
-        dt, pairs, nq = run(n2)
+    nq = max(threads, 4)
+    dt, pairs, nq = run(nq)
+    while dt < budget_s / 3 and nq < G * N:
+        nq = int(min(G * N, nq * min(8.0, max(2.0, budget_s / max(dt, 1e-3)))))
+        dt, pairs, nq = run(nq)
     tflops = 4.0 * d * pairs / dt / 1e12
     return tflops, {"queries": nq, "heads": sel, "seconds": round(dt, 3), "threads": threads,
                     "retained_pairs": pairs}
@@ -268,6 +269,9 @@ def run_tra(args, rank, world):
     from sparse_attention_video_tra_b200 import Plan, synth
     from sparse_attention_video_tra_b200.runner import WorkloadRun
     wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        wl = dataclasses.replace(wl, heads=args.heads, name=wl.name.replace(f"{wl.heads} heads", f"{args.heads} heads"))
     calls = args.calls if args.calls else (10 if args.workload == "wan720" else 1)
     run = WorkloadRun(wl, calls=calls, seed_offset=rank)
     dev_idx = torch.cuda.current_device()
@@ -383,12 +387,13 @@ def run_e2e(run, wl, calls, args, world):
     hq = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     hk = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     hv = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
-    ho = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    ho = torch.empty(shape, dtype=run.out.dtype, pin_memory=True)
     tmp = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
     plan.permute(run.q, tmp, False); hq.copy_(tmp)
     plan.permute(run.k, tmp, False); hk.copy_(tmp)
     plan.permute(run.v[0], tmp, False); hv.copy_(tmp)
-    dq, dk, dv, dn = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    dq, dk, dv = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    dn = torch.empty(shape, dtype=run.out.dtype, device="cuda")
     del tmp
 
     def step():
@@ -419,8 +424,9 @@ def run_e2e(run, wl, calls, args, world):
     secs = e0.elapsed_time(e1) / 1000.0
     val = aggregate(run.attention_flops() * calls * args.steps, secs, world) / 1e12
     nbytes = i.heads * i.N * i.d * 2
+    obytes = i.heads * i.N * i.d * run.out.element_size()
     return {"value": round(val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": nbytes * (2 + calls),
-            "d2h_bytes_per_step": nbytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3)}
+            "d2h_bytes_per_step": obytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3)}
 
 
 def main(argv=None):
@@ -431,6 +437,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="tra", choices=["tra", "reference"])
     ap.add_argument("--workload", default="wan720")
     ap.add_argument("--calls", type=int, default=0)
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -86,6 +86,7 @@ typedef enum {
 #define TRA_FLAG_TILE_W_MASK   (0xFFu << 8)
 #define TRA_FLAG_DEBUG_NO_WAIT (1u << 16)  /* test hook: pipeline waits give up at
                                               once, exercising the timeout path */
+#define TRA_FLAG_OUT_BF16      (1u << 17)  /* tra_attention writes bf16 instead of fp32 */
 
 /* everything a caller needs to size and read buffers */
 typedef struct {
@@ -136,16 +137,18 @@ TRA_API void tra_plan_destroy(tra_plan plan);
 TRA_API tra_status tra_plan_query(tra_plan plan, tra_plan_info* info);
 
 /*
- * tra_permute -- reorder bf16 rows between the natural frame-major order and
- * the padded tile-major order ("Le Pipeline TRA", Disposition Tile-Major).
- *   src, dst   device bf16, 16-byte aligned.  to_tile_major = 1: src is
- *              [heads][N][d] natural, dst is [heads][N_pad][d] tile-major with
- *              pad rows written as zeros.  to_tile_major = 0: the reverse (pad
- *              rows of src are ignored).
+ * tra_permute -- reorder rows of d elements between the natural frame-major
+ * order and the padded tile-major order ("Le Pipeline TRA", Disposition
+ * Tile-Major).
+ *   src, dst    device buffers, 16-byte aligned.  to_tile_major = 1: src is
+ *               [heads][N][d] natural, dst is [heads][N_pad][d] tile-major with
+ *               pad rows written as zeros.  to_tile_major = 0: the reverse (pad
+ *               rows of src are ignored).
+ *   elem_bytes  2 (bf16 q/k/v rows) or 4 (fp32 attention output rows)
  * src and dst must not overlap.  Asynchronous on `stream`.
  */
 TRA_API tra_status tra_permute(tra_plan plan, const void* src, void* dst, int to_tile_major,
-                       tra_stream stream);
+                       int elem_bytes, tra_stream stream);
 
 /*
  * tra_entropy -- per-query softmax entropy of the dense warm-up step
@@ -181,11 +184,14 @@ TRA_API tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void* m
  * tra_attention -- block-sparse attention with exact token masking
  * (O_i = sum over the retained keys j of softmax(q_i.k_j/sqrt d) v_j).
  * Inactive key tiles are skipped; inside listed tiles every token pair is
- * tested, so the result equals dense attention under the token mask.
+ * tested, so the result equals dense attention under the token mask.  QK^T
+ * and PV run on the tensor cores in bf16 with fp32 accumulation; P is
+ * rounded to bf16 and O is normalised by the sum of those rounded values.
  *   q, k, v    device bf16 [heads][N_pad][d] tile-major, 16-byte aligned,
  *              finite pad rows
  *   mask       the buffer written by tra_radius_and_mask for this plan
- *   out        device bf16 [heads][N_pad][d]; pad rows unspecified
+ *   out        device [heads][N_pad][d] tile-major, fp32 (bf16 when the plan
+ *              has TRA_FLAG_OUT_BF16); pad rows unspecified
  * Asynchronous on `stream`.
  */
 TRA_API tra_status tra_attention(tra_plan plan, const void* q, const void* k, const void* v,

@@ -21,7 +21,7 @@ __all__ = [
     "TraError", "PlanInfo", "Plan", "library_path", "load_library",
     "tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
     "tra_radius_and_mask", "tra_attention", "tra_plan_status", "tra_status_string",
-    "TRA_FLAG_DEBUG_NO_WAIT", "tra_flag_tile_w",
+    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "tra_flag_tile_w",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +30,7 @@ _lib = None
 
 TRA_OK = 0
 TRA_FLAG_DEBUG_NO_WAIT = 1 << 16
+TRA_FLAG_OUT_BF16 = 1 << 17
 STATUS_NAMES = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARG", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_WORKSPACE",
                 4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT", 6: "TRA_ERR_DEVICE_CHECK"}
 
@@ -97,7 +98,7 @@ def load_library() -> ctypes.CDLL:
     L.tra_plan_destroy.restype = None
     L.tra_plan_query.argtypes = [vp, ctypes.POINTER(_Info)]
     L.tra_plan_query.restype = st
-    L.tra_permute.argtypes = [vp, vp, vp, i, vp]
+    L.tra_permute.argtypes = [vp, vp, vp, i, i, vp]
     L.tra_permute.restype = st
     L.tra_entropy.argtypes = [vp, vp, vp, vp, i, vp]
     L.tra_entropy.restype = st
@@ -141,8 +142,9 @@ def tra_plan_query(plan: int) -> PlanInfo:
     return PlanInfo(**{f: getattr(info, f) for f, _ in _Info._fields_})
 
 
-def tra_permute(plan, src_ptr, dst_ptr, to_tile_major, stream=0) -> None:
-    _check("tra_permute", load_library().tra_permute(plan, src_ptr, dst_ptr, int(to_tile_major), stream))
+def tra_permute(plan, src_ptr, dst_ptr, to_tile_major, elem_bytes=2, stream=0) -> None:
+    _check("tra_permute", load_library().tra_permute(plan, src_ptr, dst_ptr, int(to_tile_major),
+                                                     int(elem_bytes), stream))
 
 
 def tra_entropy(plan, q_ptr, k_ptr, H_ptr, key_tile_stride=1, stream=0) -> None:
@@ -169,6 +171,7 @@ class Plan:
 
     def __init__(self, T, H, W, heads, d, a, b, gamma, Rt, Bmin, flags=0):
         self.handle = tra_plan_create(T, H, W, heads, d, a, b, gamma, Rt, Bmin, flags)
+        self.flags = flags
         self.info = tra_plan_query(self.handle)
         self.params = dict(T=T, H=H, W=W, heads=heads, d=d, a=a, b=b, gamma=gamma, Rt=Rt, Bmin=Bmin)
 
@@ -188,17 +191,26 @@ class Plan:
         import torch
         return (stream if stream is not None else torch.cuda.current_stream()).cuda_stream
 
-    def _rows(self, x, rows, name):
+    def _rows(self, x, rows, name, dtype=None):
         import torch
         i = self.info
-        if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.numel() != i.heads * rows * i.d:
-            raise ValueError(f"{name}: expected contiguous cuda bf16 with {i.heads}*{rows}*{i.d} elements, "
+        dtype = dtype or torch.bfloat16
+        if x.dtype != dtype or not x.is_cuda or not x.is_contiguous() or x.numel() != i.heads * rows * i.d:
+            raise ValueError(f"{name}: expected contiguous cuda {dtype} with {i.heads}*{rows}*{i.d} elements, "
                              f"got {x.dtype} {tuple(x.shape)} on {x.device}")
 
-    def new_tile_major(self, device="cuda"):
+    @property
+    def out_dtype(self):
+        import torch
+        return torch.bfloat16 if self.flags & TRA_FLAG_OUT_BF16 else torch.float32
+
+    def new_tile_major(self, device="cuda", dtype=None):
         import torch
         i = self.info
-        return torch.empty(i.heads, i.N_pad, i.d, dtype=torch.bfloat16, device=device)
+        return torch.empty(i.heads, i.N_pad, i.d, dtype=dtype or torch.bfloat16, device=device)
+
+    def new_out(self, device="cuda"):
+        return self.new_tile_major(device, self.out_dtype)
 
     def new_mask(self, device="cuda"):
         import torch
@@ -221,10 +233,14 @@ class Plan:
 
     # -- the path
     def permute(self, src, dst, to_tile_major=True, stream=None):
+        import torch
         i = self.info
-        self._rows(src, i.N if to_tile_major else i.N_pad, "src")
-        self._rows(dst, i.N_pad if to_tile_major else i.N, "dst")
-        tra_permute(self.handle, src.data_ptr(), dst.data_ptr(), 1 if to_tile_major else 0, self._stream(stream))
+        if src.dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("permute moves bf16 or fp32 rows")
+        self._rows(src, i.N if to_tile_major else i.N_pad, "src", src.dtype)
+        self._rows(dst, i.N_pad if to_tile_major else i.N, "dst", src.dtype)
+        tra_permute(self.handle, src.data_ptr(), dst.data_ptr(), 1 if to_tile_major else 0,
+                    src.element_size(), self._stream(stream))
         return dst
 
     def entropy(self, q, k, Hout, key_tile_stride=1, stream=None):
@@ -247,8 +263,9 @@ class Plan:
 
     def attention(self, q, k, v, mask, out, stream=None):
         i = self.info
-        for x, nme in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        for x, nme in ((q, "q"), (k, "k"), (v, "v")):
             self._rows(x, i.N_pad, nme)
+        self._rows(out, i.N_pad, "out", self.out_dtype)
         tra_attention(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), mask.data_ptr(), out.data_ptr(),
                       self._stream(stream))
         return out

@@ -13,7 +13,7 @@
 //              TMEM, masks, keeps the running max m and sum l (lazy rescale:
 //              O is rescaled only when the max grows by more than 2^8), writes
 //              P = 2^(S*scale - m) as bf16 into TMEM, and in the end reads O,
-//              divides by l and stores bf16 rows.
+//              divides by l and stores fp32 rows (bf16 rows on request).
 //   warp 4     TMA producer for Q and the K ring.
 //   warp 5     TMA producer for the V ring.
 //   warp 6     TMEM allocator and single-thread MMA issuer:
@@ -45,11 +45,11 @@ struct AttnCfg {
     static constexpr uint32_t COL_S = 0, COL_O = 256, COL_P = 384;
 };
 
-template <int D, int TWL>
+template <int D, int TWL, bool OUT_BF16>
 __global__ void __launch_bounds__(224, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Geom G, const uint8_t* __restrict__ mask,
-                 __nv_bfloat16* __restrict__ out)
+                 void* __restrict__ out)
 {
     using C = AttnCfg<D>;
     constexpr int TW = 1 << TWL;
@@ -264,6 +264,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tmem_wait_st();
                 }
             }
+            // P goes to the tensor core as bf16; l sums those same rounded values,
+            // so O = sum(P v) / sum(P) is an exact weighted mean of the kept v rows
             const float neg_m = -m_run;
             float lsum = 0.f;
             uint32_t pk[64];
@@ -271,8 +273,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int c = 0; c < 64; ++c) {
                 const float p0 = ex2(fmaf(s[2 * c], G.scale_log2, neg_m));
                 const float p1 = ex2(fmaf(s[2 * c + 1], G.scale_log2, neg_m));
-                lsum += p0 + p1;
                 pk[c] = pack_bf16x2(p0, p1);
+                lsum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
             }
             l += lsum;
             if (j >= 2) {
@@ -294,19 +296,27 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tc_fence_after();
                 __syncwarp();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(row0 + row) * D);
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(tmem + lane_base + C::COL_O + c * 32, v);
                     tmem_wait_ld();
-                    uint32_t o[16];
+                    if constexpr (OUT_BF16) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + (size_t)(row0 + row) * D);
+                        uint32_t o[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        o[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
+                        for (int i = 0; i < 16; ++i)
+                            o[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[c * 4 + i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                        for (int i = 0; i < 4; ++i)
+                            dst[c * 4 + i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + (size_t)(row0 + row) * D);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[c * 8 + i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                                                         __uint_as_float(v[4 * i + 2]) * inv, __uint_as_float(v[4 * i + 3]) * inv);
+                    }
                 }
             }
         }

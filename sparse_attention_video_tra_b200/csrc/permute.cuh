@@ -6,16 +6,17 @@
 // the sequence.  Natural order n = (t*H + h)*W + w ("Token Radius Attention"
 // blog post, sections 5.1 and 9.1).
 //
-// One thread moves 16 bytes; a row of d bf16 is d/8 threads.  HBM-bound.
+// One thread moves 16 bytes; a row of d elements (bf16 or fp32) is d*size/16
+// threads.  HBM-bound.
 #pragma once
 #include "tra_common.cuh"
 
 namespace tra {
 
 __global__ void __launch_bounds__(256) permute_kernel(const Geom G, const uint4* __restrict__ src,
-                                                      uint4* __restrict__ dst, int to_tile_major)
+                                                      uint4* __restrict__ dst, int to_tile_major, int elem_bytes)
 {
-    const int chunks = G.D >> 3;                     // 16-byte chunks per row
+    const int chunks = (G.D * elem_bytes) >> 4;      // 16-byte chunks per row
     const size_t total = (size_t)G.G * G.N_pad * chunks;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
          i += (size_t)gridDim.x * blockDim.x) {

@@ -64,12 +64,12 @@ bool set_smem(K kernel, int bytes)
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
-template <int D, int TWL>
+template <int D, int TWL, bool OB>
 tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                         const uint8_t* mask, __nv_bfloat16* out, cudaStream_t st)
+                         const uint8_t* mask, void* out, cudaStream_t st)
 {
     using C = tra::AttnCfg<D>;
-    auto kern = tra::attention_kernel<D, TWL>;
+    auto kern = tra::attention_kernel<D, TWL, OB>;
     if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
     kern<<<dim3(G.nQ, G.G), C::THREADS, C::SMEM, st>>>(q, k, v, G, mask, out);
     return launch_status();
@@ -88,14 +88,16 @@ tra_status run_entropy(const tra::Geom& G, const CUtensorMap& q, const CUtensorM
 
 }  // namespace
 
-extern "C" tra_status tra_permute(tra_plan plan, const void* src, void* dst, int to_tile_major, tra_stream stream)
+extern "C" tra_status tra_permute(tra_plan plan, const void* src, void* dst, int to_tile_major, int elem_bytes,
+                                  tra_stream stream)
 {
     if (!plan || !src || !dst || !aligned(src, 16) || !aligned(dst, 16)) return TRA_ERR_INVALID_ARG;
+    if (elem_bytes != 2 && elem_bytes != 4) return TRA_ERR_INVALID_ARG;
     const tra::Geom& G = plan->geom;
-    const size_t total = (size_t)G.G * G.N_pad * (G.D / 8);
+    const size_t total = (size_t)G.G * G.N_pad * (G.D * elem_bytes / 16);
     const int blocks = (int)std::min<size_t>((total + 255) / 256, 148 * 32);
     tra::permute_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(G, (const uint4*)src, (uint4*)dst,
-                                                                   to_tile_major ? 1 : 0);
+                                                                   to_tile_major ? 1 : 0, elem_bytes);
     return launch_status();
 }
 
@@ -158,17 +160,24 @@ extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k,
         return TRA_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     const uint8_t* m = (const uint8_t*)mask;
-    __nv_bfloat16* o = (__nv_bfloat16*)out;
-    const int key = G.D * 100 + G.tw_log2;
+    const int key = G.D * 100 + G.tw_log2 + ((plan->flags & TRA_FLAG_OUT_BF16) ? 10 : 0);
     switch (key) {
-        case 6402: return run_attention<64, 2>(G, mq, mk, mv, m, o, st);
-        case 6403: return run_attention<64, 3>(G, mq, mk, mv, m, o, st);
-        case 6404: return run_attention<64, 4>(G, mq, mk, mv, m, o, st);
-        case 6405: return run_attention<64, 5>(G, mq, mk, mv, m, o, st);
-        case 12802: return run_attention<128, 2>(G, mq, mk, mv, m, o, st);
-        case 12803: return run_attention<128, 3>(G, mq, mk, mv, m, o, st);
-        case 12804: return run_attention<128, 4>(G, mq, mk, mv, m, o, st);
-        case 12805: return run_attention<128, 5>(G, mq, mk, mv, m, o, st);
+        case 6402: return run_attention<64, 2, false>(G, mq, mk, mv, m, out, st);
+        case 6403: return run_attention<64, 3, false>(G, mq, mk, mv, m, out, st);
+        case 6404: return run_attention<64, 4, false>(G, mq, mk, mv, m, out, st);
+        case 6405: return run_attention<64, 5, false>(G, mq, mk, mv, m, out, st);
+        case 12802: return run_attention<128, 2, false>(G, mq, mk, mv, m, out, st);
+        case 12803: return run_attention<128, 3, false>(G, mq, mk, mv, m, out, st);
+        case 12804: return run_attention<128, 4, false>(G, mq, mk, mv, m, out, st);
+        case 12805: return run_attention<128, 5, false>(G, mq, mk, mv, m, out, st);
+        case 6412: return run_attention<64, 2, true>(G, mq, mk, mv, m, out, st);
+        case 6413: return run_attention<64, 3, true>(G, mq, mk, mv, m, out, st);
+        case 6414: return run_attention<64, 4, true>(G, mq, mk, mv, m, out, st);
+        case 6415: return run_attention<64, 5, true>(G, mq, mk, mv, m, out, st);
+        case 12812: return run_attention<128, 2, true>(G, mq, mk, mv, m, out, st);
+        case 12813: return run_attention<128, 3, true>(G, mq, mk, mv, m, out, st);
+        case 12814: return run_attention<128, 4, true>(G, mq, mk, mv, m, out, st);
+        case 12815: return run_attention<128, 5, true>(G, mq, mk, mv, m, out, st);
     }
     return TRA_ERR_UNSUPPORTED;
 }

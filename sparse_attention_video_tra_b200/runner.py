@@ -44,7 +44,7 @@ class WorkloadRun:
             self.v.append(vt)
             del vc
         del q, k, v
-        self.out = probe.new_tile_major(device)
+        self.out = probe.new_out(device)
         self.H = torch.empty(G, i.N_pad, dtype=torch.float32, device=device)
         self.mask = probe.new_mask(device)
         torch.cuda.synchronize()

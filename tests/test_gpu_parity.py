@@ -64,6 +64,13 @@ def test_permute_round_trip(c):
     assert torch.equal(back.view(torch.int16), x.view(torch.int16))
     ref = gh.to_tile_major(x, i)
     assert torch.equal(tm.view(torch.int16), ref.view(torch.int16))      # pads are zeros, rows in place
+    xf = torch.randn(i.heads, i.N, i.d, device="cuda")
+    tf = torch.full((i.heads, i.N_pad, i.d), float("nan"), device="cuda")
+    plan.permute(xf, tf, True)
+    bf = torch.empty_like(xf)
+    plan.permute(tf, bf, False)
+    torch.cuda.synchronize()
+    assert torch.equal(bf, xf) and torch.equal(tf, gh.to_tile_major(xf, i))
     assert plan.status() == 0
 
 
@@ -152,7 +159,7 @@ def test_attention_matches_oracle(c):
     mask = plan.new_mask()
     plan.radius_and_mask(gh.to_tile_major(torch.from_numpy(Hn).cuda(), i), mask)
     qt, kt, vt = (gh.to_tile_major(x, i) for x in (q, k, v))
-    out = torch.full_like(qt, float("nan"))
+    out = torch.full((G, i.N_pad, d), float("nan"), device="cuda", dtype=torch.float32)
     plan.attention(qt, kt, vt, mask, out)
     torch.cuda.synchronize()
     assert plan.status() == 0
@@ -172,10 +179,10 @@ def test_attention_special_cases(c):
     i = plan.info
     mask = plan.new_mask()
     plan.radius_and_mask(torch.zeros(G, i.N_pad, device="cuda"), mask)
-    out = torch.empty(G, i.N_pad, d, device="cuda", dtype=torch.bfloat16)
+    out = plan.new_out()
     plan.attention(gh.to_tile_major(q, i), gh.to_tile_major(k, i), gh.to_tile_major(v, i), mask, out)
     o = gh.to_natural(out, i)
-    assert torch.equal(o.view(torch.int16), v.view(torch.int16))
+    assert torch.equal(o, v.float())
     # dense
     plan = tra.Plan(T, H, W, G, d, 1.0, 60.0, 0.8, T - 1, 1)
     i = plan.info
@@ -184,7 +191,7 @@ def test_attention_special_cases(c):
     _, cnt, pairs, _ = plan.mask_views(mask)
     assert int(pairs.sum()) == G * i.N * i.N
     assert torch.all(cnt == i.n_tiles)
-    out = torch.empty(G, i.N_pad, d, device="cuda", dtype=torch.bfloat16)
+    out = plan.new_out()
     plan.attention(gh.to_tile_major(q, i), gh.to_tile_major(k, i), gh.to_tile_major(v, i), mask, out)
     o = gh.to_natural(out, i).double()
     ref = torch.nn.functional.scaled_dot_product_attention(q.double()[None], k.double()[None], v.double()[None])[0]
@@ -204,7 +211,7 @@ def test_pipeline_entropy_mask_attention(c):
     qt, kt, vt = (gh.to_tile_major(x, i) for x in (q, k, v))
     Ht = torch.empty(G, i.N_pad, device="cuda", dtype=torch.float32)
     mask = plan.new_mask()
-    out = torch.empty_like(qt)
+    out = plan.new_out()
     plan.entropy(qt, kt, Ht)
     plan.radius_and_mask(Ht, mask)
     plan.attention(qt, kt, vt, mask, out)
@@ -239,7 +246,7 @@ def test_mask_reuse_across_calls_with_fresh_v():
     qt, kt = gh.to_tile_major(q, i), gh.to_tile_major(k, i)
     for call in range(3):
         v = synth.make_v(T, H, W, G, d, 1000 + call, device="cuda")
-        out = torch.empty_like(qt)
+        out = plan.new_out()
         plan.attention(qt, kt, gh.to_tile_major(v, i), mask, out)
         ref = oracle.attention(gh.bf16_bits(q), gh.bf16_bits(k), gh.bf16_bits(v), r_o, G, (T, H, W), d, gamma, Rt)
         gh.check_attention(gh.to_natural(out, i).float().cpu().numpy().reshape(G * N, d), ref)
@@ -249,19 +256,23 @@ def test_argument_errors_on_device_calls():
     plan = _plan(CASES[0])
     i = plan.info
     x = plan.new_tile_major()
+    o = plan.new_out()
     Ht = torch.empty(i.heads, i.N_pad, device="cuda")
     mask = plan.new_mask()
     with pytest.raises(tra.TraError) as e:
         tra.tra_radius_and_mask(plan.handle, Ht.data_ptr(), mask.data_ptr(), i.mask_bytes - 1)
     assert e.value.status == 3
     with pytest.raises(tra.TraError) as e:
-        tra.tra_attention(plan.handle, x.data_ptr() + 2, x.data_ptr(), x.data_ptr(), mask.data_ptr(), x.data_ptr())
+        tra.tra_attention(plan.handle, x.data_ptr() + 2, x.data_ptr(), x.data_ptr(), mask.data_ptr(), o.data_ptr())
     assert e.value.status == 1
     with pytest.raises(tra.TraError) as e:
         tra.tra_entropy(plan.handle, x.data_ptr(), x.data_ptr(), Ht.data_ptr(), 0)
     assert e.value.status == 1
     with pytest.raises(tra.TraError) as e:
-        tra.tra_attention(plan.handle, 0, x.data_ptr(), x.data_ptr(), mask.data_ptr(), x.data_ptr())
+        tra.tra_attention(plan.handle, 0, x.data_ptr(), x.data_ptr(), mask.data_ptr(), o.data_ptr())
+    assert e.value.status == 1
+    with pytest.raises(tra.TraError) as e:
+        tra.tra_permute(plan.handle, x.data_ptr(), o.data_ptr(), 1, 3)
     assert e.value.status == 1
 
 
@@ -282,7 +293,7 @@ def test_bounded_wait_gives_up_and_context_survives():
     good.radius_and_mask(Ht, mask)
     torch.cuda.synchronize()
     assert good.status() == 0
-    out = torch.empty_like(qt)
+    out = good.new_out()
     bad.attention(qt, kt, vt, mask, out)
     torch.cuda.synchronize()
     assert bad.status() == 5
@@ -295,3 +306,27 @@ def test_bounded_wait_gives_up_and_context_survives():
     torch.cuda.synchronize()
     assert good.status() == 0
     assert torch.isfinite(gh.to_natural(out, i).float()).all()
+
+
+@pytest.mark.parametrize("c", [CASES[1], CASES[4]], ids=_ids)
+def test_attention_bf16_output(c):
+    """bf16 output: the fp32 result rounded once more; allowed error adds half a
+    bf16 ulp of the reference value (2^-9 relative) to the fp32 bound."""
+    T, H, W, G, d, gamma, Rt, Bmin, _ = c
+    N = T * H * W
+    plan = _plan(c, 1.0, math.log(0.4), flags=tra.TRA_FLAG_OUT_BF16)
+    i = plan.info
+    q, k, v = _qkv(c, 77)
+    Hn = np.random.default_rng(4).uniform(0.0, math.log(N), size=(G, N)).astype(np.float32)
+    mask = plan.new_mask()
+    plan.radius_and_mask(gh.to_tile_major(torch.from_numpy(Hn).cuda(), i), mask)
+    out = plan.new_out()
+    assert out.dtype == torch.bfloat16
+    plan.attention(*(gh.to_tile_major(x, i) for x in (q, k, v)), mask, out)
+    torch.cuda.synchronize()
+    o = gh.to_natural(out, i).double().cpu().numpy().reshape(G * N, d)
+    r_o, _, _ = oracle.radius(Hn.reshape(-1), G, (T, H, W), 1.0, math.log(0.4), gamma, Rt, Bmin)
+    ref = oracle.attention(gh.bf16_bits(q), gh.bf16_bits(k), gh.bf16_bits(v), r_o, G, (T, H, W), d, gamma, Rt)
+    err = np.abs(o - ref)
+    assert np.all(err <= gh.ATT_MAX + np.abs(ref) * 2.0 ** -9)
+    assert err.mean() <= gh.ATT_MEAN + 2.0 ** -9 * np.abs(ref).mean()
