@@ -38,6 +38,10 @@ struct EntCfg {
     static constexpr int THREADS = 192;
 };
 
+// exp2 of the elements with (index % POLY_MOD) == POLY_MOD - 1 runs on the FMA
+// pipe (degree-4 polynomial), the rest on the MUFU unit
+constexpr int POLY_MOD = 3;
+
 template <int D, int TWL>
 __global__ void __launch_bounds__(192, 2)
 entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -139,14 +143,14 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             float s[128];
             {
-                uint32_t v[32];
+                uint32_t v[4][32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    tmem_ld32(tmem + lane_base + bs * 128 + q * 32, v);
-                    tmem_wait_ld();
+                for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_base + bs * 128 + q * 32, v[q]);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(v[i]);
-                }
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(v[q][i]);
             }
             tc_fence_before();
             mbar_arrive(&s_empty[bs]);
@@ -154,12 +158,18 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 uint32_t keep[4];
                 row_keep_bits<TWL>(0, khv - 1, 0, kwv - 1, keep);
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    if (!((keep[i >> 5] >> (i & 31)) & 1u)) s[i] = -1e30f;
+                for (int i = 0; i < 128; ++i) s[i] = (keep[i >> 5] & (1u << (i & 31))) ? s[i] : -1e30f;
             }
-            float mx = s[0];
+            // four independent max chains, then combine
+            float m4[4];
 #pragma unroll
-            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+            for (int q = 0; q < 4; ++q) {
+                float a = max3(s[q * 32], s[q * 32 + 1], s[q * 32 + 2]);
+#pragma unroll
+                for (int i = 3; i < 31; i += 2) a = max3(a, s[q * 32 + i], s[q * 32 + i + 1]);
+                m4[q] = fmaxf(a, s[q * 32 + 31]);
+            }
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             const float mt = mx * c;
             if (mt > m) {
                 const float alpha = ex2(m - mt);
@@ -167,16 +177,18 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 Z *= alpha;
                 m = mt;
             }
-            float zt = 0.f, at = 0.f;
+            // eight independent partial sums keep the adds off one serial chain
+            float zt[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            float at[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 128; ++i) {
                 const float u = fmaf(s[i], c, -m);
-                const float e = ex2(u);
-                zt += e;
-                at = fmaf(e, u, at);
+                const float e = (i % POLY_MOD == POLY_MOD - 1) ? ex2_poly<4>(u) : ex2(u);
+                zt[i & 7] += e;
+                at[i & 7] = fmaf(e, u, at[i & 7]);
             }
-            Z += zt;
-            A += at;
+            Z += ((zt[0] + zt[1]) + (zt[2] + zt[3])) + ((zt[4] + zt[5]) + (zt[6] + zt[7]));
+            A += ((at[0] + at[1]) + (at[2] + at[3])) + ((at[4] + at[5]) + (at[6] + at[7]));
         }
         if (ok) {
             const float H = logf(Z) - 0.69314718055994531f * (A / Z) + corr;
