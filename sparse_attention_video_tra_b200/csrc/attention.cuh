@@ -8,23 +8,24 @@
 // against the query's per-frame half-width), so the result is exactly
 // softmax attention under the radius mask.
 //
-// One CTA per (query tile of 128 tokens, head).  352 threads:
-//   warps 0-7  softmax: query row r = TMEM lane r is shared by warps r/32 and
-//              r/32 + 4, each taking 64 of the 128 key columns.  Reads S from
-//              TMEM, masks, combines the two halves' row maxima through shared
-//              memory, keeps the running max m (lazy rescale: O is rescaled
-//              only when the max grows by more than 2^8), writes
-//              P = 2^(S*scale - m) as bf16 into TMEM, and in the end divides O
-//              by the row sum and stores the rows.
-//   warp 8     TMA producer for Q and the K ring.
-//   warp 9     TMA producer for the V ring.
-//   warp 10    TMEM allocator and single-thread MMA issuer:
-//                S[j%2] = Q K_j^T        (A, B from smem, K-major)
-//                O     += P_j V_j        (A = P from TMEM, B = V from smem, MN-major)
-//                L     += P_j 1          (B = a bf16 ones tile in smem)
-//              so the row sum L is the fp32 sum of exactly the bf16 P values
-//              the tensor core multiplied, and O / L is their weighted mean.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D), P [384,448), L [448,464).
+// One CTA per pair of query tiles (A = tile 2p, B = tile 2p+1) of one head.
+// The two tiles' key-tile lists are merged (a sorted union with per-tile
+// "listed" and "full" flags); each merged key tile is loaded once and used by
+// whichever of A and B lists it.  352 threads:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
+//              warpgroup owns query row r (TMEM lane r).  Reads S from TMEM,
+//              masks, keeps the running max m (lazy rescale: O is rescaled only
+//              when the max grows by more than 2^8) and the row sum l of the
+//              bf16-rounded P it writes back into the first 64 columns of S.
+//              The two warpgroups work on independent tiles, so one computes
+//              while the other waits for the tensor core.
+//   warp 8     TMA producer: Q_A, Q_B, then the K and V rings.
+//   warps 9,10 MMA issuers for tiles A and B (warp 9 also allocates TMEM): for
+//              each listed key tile j, S_w = Q_w K(j)^T (once PV_w of the
+//              previous tile is complete: P_w lives in S_w), then
+//              O_w += P_w(j) V(j); the two tiles progress independently.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
+// (P_A, P_B as bf16 pairs in the first 64 columns of S_A, S_B).
 #pragma once
 #include "pipeline.cuh"
 
@@ -35,38 +36,51 @@ struct AttnCfg {
     static constexpr int PANEL = 128 * 128;                 // one 64-column panel of 128 rows, bytes
     static constexpr int NP = D / 64;                       // panels per 128-row tile
     static constexpr int TILE = NP * PANEL;                 // bytes of a 128 x D bf16 tile
-    static constexpr int KST = (D == 128) ? 3 : 4;          // K ring depth
+    static constexpr int KST = (D == 128) ? 2 : 3;          // K ring depth
     static constexpr int VST = (D == 128) ? 2 : 3;          // V ring depth
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = TILE;
+    static constexpr int OFF_Q = 0;                         // Q_A, Q_B
+    static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_V = OFF_K + KST * TILE;
-    static constexpr int OFF_ONES = OFF_V + VST * TILE;     // 16 x 64 bf16 ones (2 KB)
-    static constexpr int OFF_LIST = OFF_ONES + 2048;        // decoded key tiles, uint32 [LIST_CAP]
-    static constexpr int OFF_RED = OFF_LIST + TRA_MAX_LIST_CAP * 4;   // row-max exchange [2][2][128] f32
-    static constexpr int OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
-    static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 + 2 + 1 + 1 + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
-    static constexpr int SOFTMAX_WARPS = 8;                 // two per TMEM lane quarter
-    static constexpr int WARP_K = 8, WARP_V = 9, WARP_MMA = 10;
+    static constexpr int OFF_DYN = OFF_V + VST * TILE;      // lists, half-widths, bitmaps, barriers
+    static constexpr int WARP_LOAD = 8, WARP_MMA = 9;       // MMA issuers: warps 9 (tile A), 10 (tile B)
     static constexpr int THREADS = 352;
-    static constexpr uint32_t COL_S = 0, COL_O = 256, COL_P = 384, COL_L = 448;
-    // exp2 of the P pairs with (pair % POLY_MOD) == POLY_MOD - 1 runs on the FMA
-    // pipe, the rest on the MUFU unit
-    static constexpr int POLY_MOD = 3;
 };
 
-// A listed key tile decoded once per CTA: frame (15 bits), tile row (6),
-// tile column (5), full flag (bit 31).
-__device__ __forceinline__ uint32_t pack_tile(int t, int tr, int tc, bool full)
+// TMEM columns of the S (and P) and O accumulators of query tile w = 0 (A), 1 (B)
+__device__ __forceinline__ uint32_t col_s(int w) { return w ? 128u : 0u; }
+__device__ __forceinline__ uint32_t col_o(int w) { return w ? 384u : 256u; }
+
+// Shared-memory layout after the fixed Q/K/V region; sizes depend on the plan.
+struct AttnDyn {
+    int merged, stab, bits, bars, misc, total, bw;
+    __host__ __device__ static AttnDyn make(int list_cap, int rte, int tiles_per_frame)
+    {
+        AttnDyn L;
+        // key tiles a pair of query tiles can reach: frames t-Rt' .. t+1+Rt'
+        L.bw = ((2 * rte + 2) * tiles_per_frame + 31) / 32;
+        L.merged = 0;                                               // uint32 [2 * list_cap]
+        L.stab = L.merged + 8 * list_cap;                           // uint8 [2][rte + 1][128]
+        L.bits = L.stab + ((2 * (rte + 1) * 128 + 15) & ~15);       // uint32 [5][bw]
+        L.bars = L.bits + ((5 * L.bw * 4 + 15) & ~15);              // uint64 [32]
+        L.misc = L.bars + 8 * 32;
+        L.total = L.misc + 16;
+        return L;
+    }
+};
+
+template <int D>
+inline int attn_smem_bytes(int list_cap, int rte, int tiles_per_frame)
 {
-    return (uint32_t)t | ((uint32_t)tr << 15) | ((uint32_t)tc << 21) | (full ? 0x80000000u : 0u);
+    return AttnCfg<D>::OFF_DYN + AttnDyn::make(list_cap, rte, tiles_per_frame).total + 1024;
 }
 
-__device__ __forceinline__ void named_bar(int id, int threads)
+// A merged key tile: frame (15 bits), tile row (6), tile column (5), then
+// listed-by-A (26), listed-by-B (27), full-for-A (28), full-for-B (29).
+__device__ __forceinline__ uint32_t pack_tile(int t, int tr, int tc)
 {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+    return (uint32_t)t | ((uint32_t)tr << 15) | ((uint32_t)tc << 21);
 }
+constexpr uint32_t MT_IN0 = 1u << 26, MT_FULL0 = 1u << 28;
 
 template <int D, int TWL, bool OUT_BF16>
 __global__ void __launch_bounds__(352, 1)
@@ -78,48 +92,83 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     constexpr int TW = 1 << TWL;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem + C::OFF_Q;
-    uint8_t* sK = smem + C::OFF_K;
-    uint8_t* sV = smem + C::OFF_V;
-    uint32_t* sOnes = reinterpret_cast<uint32_t*>(smem + C::OFF_ONES);
-    uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::OFF_LIST);
-    float* s_red = reinterpret_cast<float*>(smem + C::OFF_RED);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    const AttnDyn L = AttnDyn::make(G.list_cap, G.rte, G.tiles_per_frame);
+    uint8_t* dyn = smem + C::OFF_DYN;
+    uint32_t* merged = reinterpret_cast<uint32_t*>(dyn + L.merged);
+    uint8_t* s_tab = dyn + L.stab;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(dyn + L.bits);      // [5][bw]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(dyn + L.bars);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
     uint64_t* k_empty = k_full + C::KST;
     uint64_t* v_full = k_empty + C::KST;
     uint64_t* v_empty = v_full + C::VST;
-    uint64_t* s_full = v_empty + C::VST;
-    uint64_t* s_empty = s_full + 2;
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* pv_done = p_full + 1;
-    uint64_t* drain = pv_done + 1;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    uint64_t* s_full = v_empty + C::VST;     // [2]: A, B
+    uint64_t* p_full = s_full + 2;           // [2]
+    uint64_t* pv_done = p_full + 2;          // [2]
+    uint64_t* drain = pv_done + 2;           // [2]
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(dyn + L.misc);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(dyn + L.misc + 4);
+    int* s_n = reinterpret_cast<int*>(dyn + L.misc + 8);
 
-    const int tile = blockIdx.x, g = blockIdx.y;
+    const int pair = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = reinterpret_cast<const int32_t*>(mask + G.off_count)[(size_t)g * G.nQ + tile];
-    const uint16_t* glist = reinterpret_cast<const uint16_t*>(mask + G.off_list) + ((size_t)g * G.nQ + tile) * G.list_cap;
-    for (int i = tid; i < n; i += C::THREADS) {
-        const int e = glist[i];
-        int tk, trk, tck;
-        tile_coords(G, e & 0x7fff, tk, trk, tck);
-        list[i] = pack_tile(tk, trk, tck, (e & 0x8000) != 0);
-    }
-    for (int i = tid; i < 512; i += C::THREADS) sOnes[i] = 0x3F803F80u;    // bf16 1.0 pairs
-    fence_proxy_async_smem();                                              // visible to the tensor core
-    const int row0 = g * G.N_pad + tile * 128;               // first tile-major row of this tile
+    const int qa = 2 * pair, qb = 2 * pair + 1;
+    const bool hasB = qb < G.nQ;
+    const int32_t* counts = reinterpret_cast<const int32_t*>(mask + G.off_count) + (size_t)g * G.nQ;
+    const uint16_t* lists = reinterpret_cast<const uint16_t*>(mask + G.off_list) + (size_t)g * G.nQ * G.list_cap;
+    const int nA = counts[qa], nB = hasB ? counts[qb] : 0;
+    const int ta = qa / G.tiles_per_frame;
+    const int base = max(0, ta - G.rte) * G.tiles_per_frame;   // first key tile either list can hold
 
+    // ---- merge the two sorted lists: set bits, scan word counts, expand in order
+    for (int i = tid; i < 5 * L.bw; i += C::THREADS) bits[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < nA + nB; i += C::THREADS) {
+        const bool isB = i >= nA;
+        const int e = isB ? lists[(size_t)qb * G.list_cap + (i - nA)] : lists[(size_t)qa * G.list_cap + i];
+        const int bit = (e & 0x7fff) - base;
+        atomicOr(&bits[(isB ? 1 : 0) * L.bw + (bit >> 5)], 1u << (bit & 31));
+        if (e & 0x8000) atomicOr(&bits[(isB ? 3 : 2) * L.bw + (bit >> 5)], 1u << (bit & 31));
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int w0 = 0; w0 < L.bw; w0 += 32) {
+            const int w = w0 + lane;
+            const int c = w < L.bw ? __popc(bits[w] | bits[L.bw + w]) : 0;
+            int incl = c;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (w < L.bw) bits[4 * L.bw + w] = carry + incl - c;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) *s_n = carry;
+    }
+    __syncthreads();
+    for (int w = tid; w < L.bw; w += C::THREADS) {
+        const uint32_t ia = bits[w], ib = bits[L.bw + w], fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
+        uint32_t m = ia | ib;
+        int pos = (int)bits[4 * L.bw + w];
+        while (m) {
+            const int b = __ffs(m) - 1;
+            m &= m - 1;
+            int tk, trk, tck;
+            tile_coords(G, base + 32 * w + b, tk, trk, tck);
+            const uint32_t bit = 1u << b;
+            merged[pos++] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) | ((ib & bit) ? (MT_IN0 << 1) : 0u) |
+                            ((fa & bit) ? MT_FULL0 : 0u) | ((fb & bit) ? (MT_FULL0 << 1) : 0u);
+        }
+    }
     if (tid == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < C::KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
-        for (int i = 0; i < C::VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 32 * C::SOFTMAX_WARPS); }
-        mbar_init(p_full, 32 * C::SOFTMAX_WARPS);
-        mbar_init(pv_done, 1);
-        mbar_init(drain, 1);
+        for (int i = 0; i < C::KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 2); }
+        for (int i = 0; i < C::VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 2); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1); mbar_init(&drain[i], 1);
+        }
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -127,251 +176,229 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    const int n = *s_n;
+    uint8_t* sQ = smem + C::OFF_Q;
+    uint8_t* sK = smem + C::OFF_K;
+    uint8_t* sV = smem + C::OFF_V;
     const int kbase = g * G.N_pad;
-    auto key_row = [&](int j) {
-        const uint32_t e = list[j];
+    auto key_row = [&](uint32_t e) {
         return kbase + (((int)(e & 0x7fff) * G.nTh + (int)((e >> 15) & 63)) * G.nTw + (int)((e >> 21) & 31)) * 128;
     };
 
-    if (warp == C::WARP_K) {
-        // ------------------------------------------------ Q + K producer
+    if (warp == C::WARP_LOAD) {
+        // ------------------------------------------------ TMA producer: Q_A, Q_B, K and V rings
         if (lane == 0 && n > 0) {
-            prefetch_tmap(&tm_q); prefetch_tmap(&tm_k);
-            mbar_arrive_expect_tx(q_full, C::TILE);
+            prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+            mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
 #pragma unroll
-            for (int p = 0; p < C::NP; ++p) tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, row0, q_full);
-            int issued = 0;
+            for (int p = 0; p < C::NP; ++p) {
+                tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, kbase + qa * 128, q_full);
+                if (hasB) tma_load_2d(sQ + C::TILE + p * C::PANEL, &tm_q, p * 64, kbase + qb * 128, q_full);
+            }
+            int kiss = 0, viss = 0;
             for (int j = 0; j < n; ++j) {
-                const int st = j % C::KST;
-                if (j >= C::KST && !role_wait(&k_empty[st], ((j / C::KST) - 1) & 1, G.wait_ns, s_abort)) break;
-                const int y = key_row(j);
-                mbar_arrive_expect_tx(&k_full[st], C::TILE);
+                const int y = key_row(merged[j]);
+                const int ks = j % C::KST, vs = j % C::VST;
+                if (j >= C::KST && !role_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, G.wait_ns, s_abort)) break;
+                mbar_arrive_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
                 for (int p = 0; p < C::NP; ++p)
-                    tma_load_2d(sK + st * C::TILE + p * C::PANEL, &tm_k, p * 64, y, &k_full[st]);
-                ++issued;
+                    tma_load_2d(sK + ks * C::TILE + p * C::PANEL, &tm_k, p * 64, y, &k_full[ks]);
+                ++kiss;
+                if (j >= C::VST && !role_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, G.wait_ns, s_abort)) break;
+                mbar_arrive_expect_tx(&v_full[vs], C::TILE);
+#pragma unroll
+                for (int p = 0; p < C::NP; ++p)
+                    tma_load_2d(sV + vs * C::TILE + p * C::PANEL, &tm_v, p * 64, y, &v_full[vs]);
+                ++viss;
             }
             // copies still in flight must land before the CTA exits
             mbar_wait(q_full, 0, G.drain_ns);
-            for (int j = max(0, issued - C::KST); j < issued; ++j)
-                mbar_wait(&k_full[j % C::KST], (j / C::KST) & 1, G.drain_ns);
+            for (int j = max(0, kiss - C::KST); j < kiss; ++j) mbar_wait(&k_full[j % C::KST], (j / C::KST) & 1, G.drain_ns);
+            for (int j = max(0, viss - C::VST); j < viss; ++j) mbar_wait(&v_full[j % C::VST], (j / C::VST) & 1, G.drain_ns);
         }
-    } else if (warp == C::WARP_V) {
-        // ------------------------------------------------ V producer
-        if (lane == 0 && n > 0) {
-            prefetch_tmap(&tm_v);
-            int issued = 0;
-            for (int j = 0; j < n; ++j) {
-                const int st = j % C::VST;
-                if (j >= C::VST && !role_wait(&v_empty[st], ((j / C::VST) - 1) & 1, G.wait_ns, s_abort)) break;
-                const int y = key_row(j);
-                mbar_arrive_expect_tx(&v_full[st], C::TILE);
-#pragma unroll
-                for (int p = 0; p < C::NP; ++p)
-                    tma_load_2d(sV + st * C::TILE + p * C::PANEL, &tm_v, p * 64, y, &v_full[st]);
-                ++issued;
-            }
-            for (int j = max(0, issued - C::VST); j < issued; ++j)
-                mbar_wait(&v_full[j % C::VST], (j / C::VST) & 1, G.drain_ns);
-        }
-    } else if (warp == C::WARP_MMA) {
-        // ------------------------------------------------ MMA issuer
-        // order: QK_0, then for each j: QK_{j+1} (as soon as its S buffer is
-        // free), PV_j (once P_j is written), so S is ready ahead of the softmax
+    } else if (warp >= C::WARP_MMA) {
+        // ------------------------------------------------ MMA issuers, one per query tile
+        // Issuing tcgen05.mma occupies the issuing thread about as long as the
+        // tensor core runs it, so each query tile w gets its own issuer; both walk
+        // the merged list in order.  For a tile w lists: S_w = Q_w K^T (once its
+        // previous PV is complete: P_w lives in S_w), then O_w += P_w V.  Either
+        // way it releases the K and V ring stages (two arrivals per occupant): a
+        // commit after its MMAs, or a plain arrive once the tile has landed.
+        const int w = warp - C::WARP_MMA;
         if (lane == 0 && n > 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
-            constexpr uint32_t IDESC_L = idesc_bf16_f32(128, 16, false);
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sOa = smem_u32(sOnes);
-            auto issue_qk = [&](int j) -> bool {
-                const int ks = j % C::KST;
-                if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) return false;
-                if (j >= 2 && !role_wait(&s_empty[j & 1], ((j - 2) >> 1) & 1, G.wait_ns, s_abort)) return false;
+            const uint32_t sQa = smem_u32(sQ) + w * C::TILE, sKa = smem_u32(sK), sVa = smem_u32(sV);
+            const uint32_t in_bit = MT_IN0 << w;
+            bool ok = role_wait(q_full, 0, G.wait_ns, s_abort);
+            int cnt = 0;
+            for (int j = 0; ok && j < n; ++j) {
+                const bool uses = (merged[j] & in_bit) != 0;
+                const int ks = j % C::KST, vs = j % C::VST;
+                if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                if (!uses) {
+                    mbar_arrive(&k_empty[ks]);
+                    if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                    mbar_arrive(&v_empty[vs]);
+                    continue;
+                }
+                if (cnt > 0 && !role_wait(&pv_done[w], (cnt - 1) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
-                    mma_ss(tmem + C::COL_S + (j & 1) * 128, smem_desc_sw128(sQa + off, 16, 1024),
+                    mma_ss(tmem + col_s(w), smem_desc_sw128(sQa + off, 16, 1024),
                            smem_desc_sw128(sKa + ks * C::TILE + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&s_full[j & 1]);
+                mma_commit(&s_full[w]);
                 mma_commit(&k_empty[ks]);
-                return true;
-            };
-            auto issue_pv = [&](int i) -> bool {
-                const int vs = i % C::VST;
-                if (!role_wait(p_full, i & 1, G.wait_ns, s_abort)) return false;
-                if (!role_wait(&v_full[vs], (i / C::VST) & 1, G.wait_ns, s_abort)) return false;
+                if (!role_wait(&p_full[w], cnt & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a_t = tmem + C::COL_P + kk * 8;
-                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts(tmem + C::COL_O, a_t, smem_desc_sw128(sVa + vs * C::TILE + kk * 2048, C::PANEL, 1024),
-                           IDESC_PV, acc);
-                    mma_ts(tmem + C::COL_L, a_t, smem_desc_sw128(sOa + (kk & 3) * 32, 16, 1024), IDESC_L, acc);
-                }
-                mma_commit(pv_done);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + col_o(w), tmem + col_s(w) + kk * 8,
+                           smem_desc_sw128(sVa + vs * C::TILE + kk * 2048, C::PANEL, 1024), IDESC_PV,
+                           (cnt > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&pv_done[w]);
                 mma_commit(&v_empty[vs]);
-                return true;
-            };
-            bool ok = role_wait(q_full, 0, G.wait_ns, s_abort) && issue_qk(0);
-            for (int j = 0; ok && j < n; ++j) {
-                if (j + 1 < n && !issue_qk(j + 1)) { ok = false; break; }
-                if (!issue_pv(j)) { ok = false; break; }
+                ++cnt;
             }
             // every issued MMA must finish before TMEM is freed
-            mma_commit(drain);
-            mbar_wait(drain, 0, G.drain_ns);
+            mma_commit(&drain[w]);
+            mbar_wait(&drain[w], 0, G.drain_ns);
         }
     } else {
         // ------------------------------------------------ softmax / epilogue (warps 0-7)
-        // warp w and warp w+4 share TMEM lanes 32*(w%4) .. +31 (query rows);
-        // half h = w/4 takes key columns [64h, 64h+64) and O columns [h*D/2, (h+1)*D/2)
-        const int quarter = warp & 3, half = warp >> 2;
-        const int row = quarter * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const int w = warp >> 2;                             // 0: tile A, 1: tile B
+        const int row = tid & 127;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t colS = col_s(w), colO = col_o(w);
+        const int qt = w ? qb : qa;
+        const bool active = w == 0 || hasB;
         int tq, trq, tcq;
-        tile_coords(G, tile, tq, trq, tcq);
+        tile_coords(G, active ? qt : qa, tq, trq, tcq);
         const int hq = trq * G.th + (row >> TWL);
         const int wq = tcq * TW + (row & (TW - 1));
-        const bool qvalid = hq < G.H && wq < G.W;
-        const int rq = qvalid ? reinterpret_cast<const int32_t*>(mask + G.off_radius)[row0 + row] : -1;
+        const bool qvalid = active && hq < G.H && wq < G.W;
+        const int rq = qvalid ? reinterpret_cast<const int32_t*>(mask + G.off_radius)[kbase + qt * 128 + row] : -1;
+        uint8_t* my_tab = s_tab + w * (G.rte + 1) * 128;
+        for (int dl = 0; dl <= G.rte; ++dl)
+            my_tab[dl * 128 + row] = (uint8_t)(qvalid ? min(halfwidth(rq, G.g[dl]), 255) : 0);
         const float sc = G.scale_log2;
+        const uint32_t in_bit = MT_IN0 << w, full_bit = MT_FULL0 << w;
 
-        float m_run = -1e30f;
+        float m_run = -1e30f, l = 0.f;
+        int k = 0;                                           // tiles processed by this query tile
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const uint32_t e = list[j];
+        for (int j = 0; active && j < n; ++j) {
+            const uint32_t e = merged[j];
+            if (!(e & in_bit)) continue;
             const int tk = (int)(e & 0x7fff), trk = (int)((e >> 15) & 63), tck = (int)((e >> 21) & 31);
             const int h0 = trk * G.th, w0 = tck * TW;
             const int khv = min(G.th, G.H - h0), kwv = min(TW, G.W - w0);
-            const bool full = (e >> 31) != 0;
+            const bool full = (e & full_bit) != 0;
             const bool need_mask = !full || khv < G.th || kwv < TW;
-            uint32_t keep[2] = {~0u, ~0u};
+            uint32_t keep[4] = {~0u, ~0u, ~0u, ~0u};
             if (need_mask) {
-                const int s = full ? 1 << 20 : (qvalid ? halfwidth(rq, G.g[abs(tk - tq)]) : -1);
+                const int s = full ? 1 << 20 : (int)my_tab[abs(tk - tq) * 128 + row];
                 int a_lo = max(0, hq - s - h0), a_hi = min(khv - 1, hq + s - h0);
                 const int b_lo = max(0, wq - s - w0), b_hi = min(kwv - 1, wq + s - w0);
                 if (!qvalid) { a_lo = 1; a_hi = 0; }
-                uint32_t k4[4];
-                row_keep_bits<TWL>(a_lo, a_hi, b_lo, b_hi, k4);
-                keep[0] = half ? k4[2] : k4[0];
-                keep[1] = half ? k4[3] : k4[1];
+                row_keep_bits<TWL>(a_lo, a_hi, b_lo, b_hi, keep);
             }
 
-            const bool got = role_wait(&s_full[j & 1], (j >> 1) & 1, G.wait_ns, s_abort);
+            const bool got = role_wait(&s_full[w], k & 1, G.wait_ns, s_abort);
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
             tc_fence_after();
             __syncwarp();
-            float s[64];
+            float s[128];
             {
-                uint32_t v[2][32];
+                uint32_t v[4][32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    tmem_ld32(tmem + lane_base + C::COL_S + (j & 1) * 128 + half * 64 + c * 32, v[c]);
+                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + c * 32, v[c]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[c][i]);
             }
-            tc_fence_before();
-            mbar_arrive(&s_empty[j & 1]);
-
             if (need_mask) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) s[c] = (keep[c >> 5] & (1u << (c & 31))) ? s[c] : -INFINITY;
+                for (int c = 0; c < 128; ++c) s[c] = (keep[c >> 5] & (1u << (c & 31))) ? s[c] : -INFINITY;
             }
             float m4[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                float a = max3(s[q * 16], s[q * 16 + 1], s[q * 16 + 2]);
+                float a = max3(s[q * 32], s[q * 32 + 1], s[q * 32 + 2]);
 #pragma unroll
-                for (int i = 3; i < 15; i += 2) a = max3(a, s[q * 16 + i], s[q * 16 + i + 1]);
-                m4[q] = fmaxf(a, s[q * 16 + 15]);
+                for (int i = 3; i < 31; i += 2) a = max3(a, s[q * 32 + i], s[q * 32 + i + 1]);
+                m4[q] = fmaxf(a, s[q * 32 + 31]);
             }
-            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // combine the two halves of the row
-            s_red[((j & 1) * 2 + half) * 128 + row] = mx;
-            named_bar(1 + quarter, 64);
-            mx = fmaxf(mx, s_red[((j & 1) * 2 + (half ^ 1)) * 128 + row]);
-            const float m_tile = mx * sc;
+            const float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
             const bool need = m_tile > m_run + 8.0f;
             float alpha = 1.f;
             if (need) { alpha = ex2(m_run - m_tile); m_run = m_tile; }
-            const bool rescale = j > 0 && __any_sync(0xffffffffu, need);
-
+            l *= alpha;
+            const bool rescale = k > 0 && __any_sync(0xffffffffu, need);
             const float neg_m = -m_run;
-            uint32_t pk[32];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float x0 = fmaf(s[2 * c], sc, neg_m);
-                const float x1 = fmaf(s[2 * c + 1], sc, neg_m);
-                float p0, p1;
-                if ((c % C::POLY_MOD) == C::POLY_MOD - 1) { p0 = ex2_poly<3>(x0); p1 = ex2_poly<3>(x1); }
-                else { p0 = ex2(x0); p1 = ex2(x1); }
-                pk[c] = pack_bf16x2(p0, p1);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int e2 = c * 16 + i;                 // pair index
+                    const float x0 = fmaf(s[2 * e2], sc, neg_m);
+                    const float x1 = fmaf(s[2 * e2 + 1], sc, neg_m);
+                    pk[i] = pack_bf16x2(ex2(x0), ex2(x1));
+                    // the row sum adds exactly the bf16 values the tensor core will use
+                    ls[i & 3] += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+                }
+                tmem_st16(tmem + lane_base + colS + c * 16, pk);
             }
-            // PV_{j-1} must be done: it reads P (single buffer) and writes O and L
-            if (j > 0) {
-                const bool done = role_wait(pv_done, (j - 1) & 1, G.wait_ns, s_abort);
-                if (__any_sync(0xffffffffu, !done)) { ok = false; break; }
-            }
-            tc_fence_after();
-            __syncwarp();
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            // O_w is complete up to tile k-1 (the QK for this tile waited for that
+            // PV); rescale it before PV of this tile is issued (after p_full)
             if (rescale) {
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
-                    const uint32_t col = C::COL_O + half * (D / 2) + c * 32;
-                    tmem_ld32(tmem + lane_base + col, v);
+                    tmem_ld32(tmem + lane_base + colO + c * 32, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st32(tmem + lane_base + col, v);
-                }
-                if (half == 0) {
-                    uint32_t v[16];
-                    tmem_ld16(tmem + lane_base + C::COL_L, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st16(tmem + lane_base + C::COL_L, v);
+                    tmem_st32(tmem + lane_base + colO + c * 32, v);
                 }
             }
-            tmem_st32(tmem + lane_base + C::COL_P + half * 32, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[w]);
+            ++k;
         }
-        if (ok && n > 0) {
-            ok = role_wait(pv_done, (n - 1) & 1, G.wait_ns, s_abort);
+        if (ok && k > 0) {
+            ok = role_wait(&pv_done[w], (k - 1) & 1, G.wait_ns, s_abort);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
                 __syncwarp();
-                uint32_t lv[16];
-                tmem_ld16(tmem + lane_base + C::COL_L, lv);
-                tmem_wait_ld();
-                const float l = __uint_as_float(lv[0]);
                 const float inv = l > 0.f ? 1.f / l : 0.f;
+                const size_t orow = (size_t)(kbase + qt * 128 + row) * D;
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
-                    const int col = half * (D / 2) + c * 32;
-                    tmem_ld32(tmem + lane_base + C::COL_O + col, v);
+                    tmem_ld32(tmem + lane_base + colO + c * 32, v);
                     tmem_wait_ld();
                     if constexpr (OUT_BF16) {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + (size_t)(row0 + row) * D + col);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + orow + c * 32);
                         uint32_t o[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             o[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
                     } else {
-                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + (size_t)(row0 + row) * D + col);
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + orow + c * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             dst[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,

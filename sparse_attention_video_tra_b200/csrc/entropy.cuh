@@ -14,10 +14,13 @@
 // a multiple of s and adds ln(N / |S|) (host-computed) so that a uniform
 // distribution still reads ln N.
 //
-// One CTA per (query tile of 128 tokens, head), two CTAs per SM.  192 threads:
-//   warps 0-3 statistics (thread i = query row i = TMEM lane i),
-//   warp 4 TMA producer (Q, then the K ring), warp 5 TMEM allocator + MMA
-//   issuer (S[j%2] = Q K_j^T, two 128-column fp32 buffers).
+// One CTA per pair of query tiles (A = 2p, B = 2p+1) of one head; every K tile
+// is loaded once and multiplied with both.  352 threads:
+//   warps 0-3 statistics of tile A, warps 4-7 of tile B (thread r = query row
+//   r = TMEM lane r); warp 8 TMA producer (Q_A, Q_B, then the K ring); warps 9
+//   and 10 MMA issuers for tiles A and B (warp 9 also allocates TMEM):
+//   S_w[j%2] = Q_w K_j^T, two 128-column fp32 buffers per query tile.
+// TMEM columns: S_A[0] [0,128), S_A[1] [128,256), S_B[0] [256,384), S_B[1] [384,512).
 #pragma once
 #include "pipeline.cuh"
 
@@ -28,22 +31,23 @@ struct EntCfg {
     static constexpr int PANEL = 128 * 128;
     static constexpr int NP = D / 64;
     static constexpr int TILE = NP * PANEL;
-    static constexpr int KST = (D == 128) ? 2 : 3;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = TILE;
+    static constexpr int KST = (D == 128) ? 4 : 8;
+    static constexpr int OFF_Q = 0;                     // Q_A, Q_B
+    static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_BAR = OFF_K + KST * TILE;
-    static constexpr int NBAR = 1 + 2 * KST + 4 + 1;
+    static constexpr int NBAR = 1 + 2 * KST + 8 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 352;
+    static constexpr int WARP_LOAD = 8, WARP_MMA = 9;     // MMA issuers: warps 9 (tile A), 10 (tile B)
 };
 
-// exp2 of the elements with (index % POLY_MOD) == POLY_MOD - 1 runs on the FMA
-// pipe (degree-4 polynomial), the rest on the MUFU unit
-constexpr int POLY_MOD = 3;
+// exp2 of the elements with (index % ENT_POLY_MOD) == ENT_POLY_MOD - 1 runs on
+// the FMA pipe (degree-4 polynomial), the rest on the MUFU unit
+constexpr int ENT_POLY_MOD = 4;
 
 template <int D, int TWL>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(352, 1)
 entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const Geom G, int stride, float corr, float* __restrict__ Hout)
 {
@@ -57,36 +61,42 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
     uint64_t* k_empty = k_full + C::KST;
-    uint64_t* s_full = k_empty + C::KST;
-    uint64_t* s_empty = s_full + 2;
-    uint64_t* drain = s_empty + 2;
+    uint64_t* s_full = k_empty + C::KST;     // [w * 2 + buffer]
+    uint64_t* s_empty = s_full + 4;          // [w * 2 + buffer]
+    uint64_t* drain = s_empty + 4;           // [2]
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
-    const int tile = blockIdx.x, g = blockIdx.y;
+    const int pair = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qa = 2 * pair, qb = 2 * pair + 1;
+    const bool hasB = qb < G.nQ;
     const int n = (G.nQ + stride - 1) / stride;              // key tiles visited
-    const int row0 = g * G.N_pad + tile * 128;
+    const int kbase = g * G.N_pad;
 
     if (tid == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < C::KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 128); }
-        mbar_init(drain, 1);
+        for (int i = 0; i < C::KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 2); }
+        for (int i = 0; i < 4; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 128); }
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *s_abort = 0;
         fence_barrier_init();
     }
-    if (warp == 5) { tmem_alloc(s_tmem, 256); tmem_relinquish(); }
+    if (warp == C::WARP_MMA) { tmem_alloc(s_tmem, 512); tmem_relinquish(); }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 4) {
+    if (warp == C::WARP_LOAD) {
         if (lane == 0) {
             prefetch_tmap(&tm_q); prefetch_tmap(&tm_k);
-            mbar_arrive_expect_tx(q_full, C::TILE);
+            mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
 #pragma unroll
-            for (int p = 0; p < C::NP; ++p) tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, row0, q_full);
+            for (int p = 0; p < C::NP; ++p) {
+                tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, kbase + qa * 128, q_full);
+                if (hasB) tma_load_2d(sQ + C::TILE + p * C::PANEL, &tm_q, p * 64, kbase + qb * 128, q_full);
+            }
             int issued = 0;
             for (int j = 0; j < n; ++j) {
                 const int st = j % C::KST;
@@ -94,49 +104,56 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 mbar_arrive_expect_tx(&k_full[st], C::TILE);
 #pragma unroll
                 for (int p = 0; p < C::NP; ++p)
-                    tma_load_2d(sK + st * C::TILE + p * C::PANEL, &tm_k, p * 64, g * G.N_pad + j * stride * 128,
-                                &k_full[st]);
+                    tma_load_2d(sK + st * C::TILE + p * C::PANEL, &tm_k, p * 64, kbase + j * stride * 128, &k_full[st]);
                 ++issued;
             }
             mbar_wait(q_full, 0, G.drain_ns);
             for (int j = max(0, issued - C::KST); j < issued; ++j)
                 mbar_wait(&k_full[j % C::KST], (j / C::KST) & 1, G.drain_ns);
         }
-    } else if (warp == 5) {
+    } else if (warp >= C::WARP_MMA) {
+        // One MMA issuer per query tile (issuing tcgen05.mma occupies the thread
+        // about as long as the tensor core runs it): S_w[j%2] = Q_w K_j^T once
+        // K_j has landed and the softmax of tile j-2 has released that buffer.
+        // Each issuer's commit is one of the two arrivals that free a K stage.
+        const int w = warp - C::WARP_MMA;
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false);
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+            const uint32_t sQa = smem_u32(sQ) + w * C::TILE, sKa = smem_u32(sK);
+            const bool active = w == 0 || hasB;
             bool ok = role_wait(q_full, 0, G.wait_ns, s_abort);
             for (int j = 0; ok && j < n; ++j) {
-                const int ks = j % C::KST;
+                const int ks = j % C::KST, b = j & 1;
                 if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) break;
-                if (j >= 2 && !role_wait(&s_empty[j & 1], ((j - 2) >> 1) & 1, G.wait_ns, s_abort)) break;
+                if (!active) { mbar_arrive(&k_empty[ks]); continue; }
+                if (j >= 2 && !role_wait(&s_empty[w * 2 + b], ((j - 2) >> 1) & 1, G.wait_ns, s_abort)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
-                    mma_ss(tmem + (j & 1) * 128, smem_desc_sw128(sQa + off, 16, 1024),
+                    mma_ss(tmem + (w * 2 + b) * 128, smem_desc_sw128(sQa + off, 16, 1024),
                            smem_desc_sw128(sKa + ks * C::TILE + off, 16, 1024), IDESC, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&s_full[j & 1]);
+                mma_commit(&s_full[w * 2 + b]);
                 mma_commit(&k_empty[ks]);
             }
-            mma_commit(drain);
-            mbar_wait(drain, 0, G.drain_ns);
+            mma_commit(&drain[w]);
+            mbar_wait(&drain[w], 0, G.drain_ns);
         }
     } else {
-        const int row = tid;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int w = warp >> 2;
+        const int row = tid & 127;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const float c = G.scale_log2;
         float m = -1e30f, Z = 0.f, A = 0.f;
-        bool ok = true;
-        for (int j = 0; j < n; ++j) {
+        bool ok = w == 0 || hasB;
+        for (int j = 0; ok && j < n; ++j) {
             const int kb = j * stride;
             int tk, trk, tck;
             tile_coords(G, kb, tk, trk, tck);
             const int khv = min(G.th, G.H - trk * G.th), kwv = min(TW, G.W - tck * TW);
             const bool edge = khv < G.th || kwv < TW;
-            const int bs = j & 1;
+            const int bs = w * 2 + (j & 1);
             const bool got = role_wait(&s_full[bs], (j >> 1) & 1, G.wait_ns, s_abort);
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
             tc_fence_after();
@@ -183,7 +200,7 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < 128; ++i) {
                 const float u = fmaf(s[i], c, -m);
-                const float e = (i % POLY_MOD == POLY_MOD - 1) ? ex2_poly<4>(u) : ex2(u);
+                const float e = (i % ENT_POLY_MOD == ENT_POLY_MOD - 1) ? ex2_poly<4>(u) : ex2(u);
                 zt[i & 7] += e;
                 at[i & 7] = fmaf(e, u, at[i & 7]);
             }
@@ -192,14 +209,14 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         if (ok) {
             const float H = logf(Z) - 0.69314718055994531f * (A / Z) + corr;
-            Hout[row0 + row] = H;
+            Hout[kbase + (w ? qb : qa) * 128 + row] = H;
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 

@@ -36,6 +36,25 @@ __device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// For event-driven issuers that poll several barriers: returns false (and
+// raises the abort flag and the error word) once no progress has been made
+// for limit_ns, or as soon as another role has aborted.
+__device__ __forceinline__ bool poll_alive(uint64_t& t_last, bool progress, uint64_t limit_ns, volatile int* abort_flag)
+{
+    if (progress) {
+        t_last = globaltimer_ns();
+        return true;
+    }
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t_last > limit_ns) {
+        *abort_flag = 1;
+        atomicOr(&g_tra_error, TRA_ERRBIT_TIMEOUT);
+        return false;
+    }
+    __nanosleep(32);
+    return true;
+}
+
 // Keep-bits of one query row inside a key tile, as four 32-column words.
 // Key (a, b) of the tile (a = key row, b = key column) is kept iff
 // a_lo <= a <= a_hi and b_lo <= b <= b_hi.

@@ -64,14 +64,19 @@ bool set_smem(K kernel, int bytes)
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+// largest dynamic shared memory a CTA may use on sm_100
+constexpr int kMaxSmem = 232448;
+
 template <int D, int TWL, bool OB>
 tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                          const uint8_t* mask, void* out, cudaStream_t st)
 {
     using C = tra::AttnCfg<D>;
     auto kern = tra::attention_kernel<D, TWL, OB>;
-    if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
-    kern<<<dim3(G.nQ, G.G), C::THREADS, C::SMEM, st>>>(q, k, v, G, mask, out);
+    const int smem = tra::attn_smem_bytes<D>(G.list_cap, G.rte, G.tiles_per_frame);
+    if (smem > kMaxSmem) return TRA_ERR_UNSUPPORTED;
+    if (!set_smem(kern, smem)) return TRA_ERR_CUDA;
+    kern<<<dim3((G.nQ + 1) / 2, G.G), C::THREADS, smem, st>>>(q, k, v, G, mask, out);
     return launch_status();
 }
 
@@ -82,7 +87,7 @@ tra_status run_entropy(const tra::Geom& G, const CUtensorMap& q, const CUtensorM
     using C = tra::EntCfg<D>;
     auto kern = tra::entropy_kernel<D, TWL>;
     if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
-    kern<<<dim3(G.nQ, G.G), C::THREADS, C::SMEM, st>>>(q, k, G, stride, corr, H);
+    kern<<<dim3((G.nQ + 1) / 2, G.G), C::THREADS, C::SMEM, st>>>(q, k, G, stride, corr, H);
     return launch_status();
 }
 

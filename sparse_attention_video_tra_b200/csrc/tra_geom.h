@@ -7,7 +7,8 @@
 #define TRA_MAX_TILES_H 64           // tile rows per frame the mask kernel handles
 #define TRA_MAX_LIST_ROWS 4096       // (2Rt'+1) * tile rows per frame
 #define TRA_MAX_R_CAP (1 << 20)
-#define TRA_MAX_LIST_CAP 4096         // key tiles listed per query tile
+#define TRA_MAX_LIST_CAP 2048         // key tiles listed per query tile
+#define TRA_MAX_HW 256                // largest H and W (half-widths kept as bytes)
 #define TRA_ERRBIT_TIMEOUT 1u
 #define TRA_ERRBIT_CHECK 2u
 

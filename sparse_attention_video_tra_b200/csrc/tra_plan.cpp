@@ -49,6 +49,7 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     if (d != 64 && d != 128) return TRA_ERR_UNSUPPORTED;
     if (flags & ~(TRA_FLAG_TILE_W_MASK | TRA_FLAG_DEBUG_NO_WAIT | TRA_FLAG_OUT_BF16)) return TRA_ERR_INVALID_ARG;
 
+    if (H > TRA_MAX_HW || W > TRA_MAX_HW) return TRA_ERR_UNSUPPORTED;
     const int rte = Rt < T - 1 ? Rt : T - 1;
     if (rte > TRA_MAX_RT_EFF) return TRA_ERR_UNSUPPORTED;
 
