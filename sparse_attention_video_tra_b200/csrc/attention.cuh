@@ -11,12 +11,15 @@
 // One CTA per pair of query tiles (A = tile 2p, B = tile 2p+1) of one head.
 // The two tiles' key-tile lists are merged (a sorted union with per-tile
 // "listed" and "full" flags); each merged key tile is loaded once and used by
-// whichever of A and B lists it.  352 threads:
+// whichever of A and B lists it.  384 threads:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
 //              warpgroup owns query row r (TMEM lane r).  Reads S from TMEM,
-//              masks, keeps the running max m (lazy rescale: O is rescaled only
-//              when the max grows by more than 2^8) and the row sum l of the
-//              bf16-rounded P it writes back into the first 64 columns of S.
+//              applies the token mask as an additive 0 / -inf bias (per key
+//              column and key row of the tile), keeps the running max m (lazy
+//              rescale: O is rescaled only when the max grows by more than
+//              2^8) and the row sum l of the bf16-rounded P it writes back into
+//              the first 64 columns of S.  Scale, bias and row sum use packed
+//              fp32x2 arithmetic.
 //              The two warpgroups work on independent tiles, so one computes
 //              while the other waits for the tensor core.
 //   warp 8     TMA producer: Q_A, Q_B, then the K and V rings.
@@ -24,6 +27,8 @@
 //              each listed key tile j, S_w = Q_w K(j)^T (once PV_w of the
 //              previous tile is complete: P_w lives in S_w), then
 //              O_w += P_w(j) V(j); the two tiles progress independently.
+//   warp 11    idle (completes the third warpgroup for register rebalancing:
+//              the softmax warpgroups run with 216 registers, warps 8-11 with 72).
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 // (P_A, P_B as bf16 pairs in the first 64 columns of S_A, S_B).
 #pragma once
@@ -43,7 +48,10 @@ struct AttnCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE;
     static constexpr int OFF_DYN = OFF_V + VST * TILE;      // lists, half-widths, bitmaps, barriers
     static constexpr int WARP_LOAD = 8, WARP_MMA = 9;       // MMA issuers: warps 9 (tile A), 10 (tile B)
-    static constexpr int THREADS = 352;
+    static constexpr int THREADS = 384;                     // warp 11 only completes warpgroup 2
+    // registers after rebalancing: softmax warpgroups 0, 1 and warpgroup 2
+    // (384 x 168 at launch = 2 x 128 x 216 + 128 x 72)
+    static constexpr int REGS_SOFTMAX = 216, REGS_OTHER = 72;
 };
 
 // TMEM columns of the S (and P) and O accumulators of query tile w = 0 (A), 1 (B)
@@ -83,7 +91,7 @@ __device__ __forceinline__ uint32_t pack_tile(int t, int tr, int tc)
 constexpr uint32_t MT_IN0 = 1u << 26, MT_FULL0 = 1u << 28;
 
 template <int D, int TWL, bool OUT_BF16>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Geom G, const uint8_t* __restrict__ mask,
                  void* __restrict__ out)
@@ -110,6 +118,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(dyn + L.misc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(dyn + L.misc + 4);
     int* s_n = reinterpret_cast<int*>(dyn + L.misc + 8);
+    int* s_lock = reinterpret_cast<int*>(dyn + L.misc + 12);
 
     const int pair = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -170,6 +179,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1); mbar_init(&drain[i], 1);
         }
         *s_abort = 0;
+        *s_lock = 0;
         fence_barrier_init();
     }
     if (warp == C::WARP_MMA) { tmem_alloc(s_tmem, 512); tmem_relinquish(); }
@@ -185,7 +195,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return kbase + (((int)(e & 0x7fff) * G.nTh + (int)((e >> 15) & 63)) * G.nTw + (int)((e >> 21) & 31)) * 128;
     };
 
-    if (warp == C::WARP_LOAD) {
+    if (warp >= C::WARP_LOAD) {
+      regs_dec<C::REGS_OTHER>();
+      if (warp == C::WARP_LOAD) {
         // ------------------------------------------------ TMA producer: Q_A, Q_B, K and V rings
         if (lane == 0 && n > 0) {
             prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
@@ -217,7 +229,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int j = max(0, kiss - C::KST); j < kiss; ++j) mbar_wait(&k_full[j % C::KST], (j / C::KST) & 1, G.drain_ns);
             for (int j = max(0, viss - C::VST); j < viss; ++j) mbar_wait(&v_full[j % C::VST], (j / C::VST) & 1, G.drain_ns);
         }
-    } else if (warp >= C::WARP_MMA) {
+      } else if (warp == C::WARP_MMA || warp == C::WARP_MMA + 1) {
         // ------------------------------------------------ MMA issuers, one per query tile
         // Issuing tcgen05.mma occupies the issuing thread about as long as the
         // tensor core runs it, so each query tile w gets its own issuer; both walk
@@ -244,6 +256,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     continue;
                 }
                 if (cnt > 0 && !role_wait(&pv_done[w], (cnt - 1) & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -253,8 +266,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 mma_commit(&s_full[w]);
                 mma_commit(&k_empty[ks]);
+                issue_unlock(s_lock);
                 if (!role_wait(&p_full[w], cnt & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -263,13 +278,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                            (cnt > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&pv_done[w]);
                 mma_commit(&v_empty[vs]);
+                issue_unlock(s_lock);
                 ++cnt;
             }
             // every issued MMA must finish before TMEM is freed
             mma_commit(&drain[w]);
             mbar_wait(&drain[w], 0, G.drain_ns);
         }
+      }
     } else {
+        regs_inc<C::REGS_SOFTMAX>();
         // ------------------------------------------------ softmax / epilogue (warps 0-7)
         const int w = warp >> 2;                             // 0: tile A, 1: tile B
         const int row = tid & 127;
@@ -289,7 +307,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float sc = G.scale_log2;
         const uint32_t in_bit = MT_IN0 << w, full_bit = MT_FULL0 << w;
 
-        float m_run = -1e30f, l = 0.f;
+        // m_run: the log2-domain maximum P is taken relative to (anchored at the
+        // first kept maximum, raised lazily when a tile exceeds it by 2^8);
+        // l: the sum of the bf16-rounded P values, in the same frame.
+        float m_run = 0.f, l = 0.f;
+        const f2_t sc2 = f2_pack(sc, sc);
+        constexpr int KR = 128 >> TWL;                       // key rows of a tile
+        constexpr int CP = TW / 2;                           // column pairs of a key row
         int k = 0;                                           // tiles processed by this query tile
         bool ok = true;
         for (int j = 0; active && j < n; ++j) {
@@ -299,77 +323,94 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int h0 = trk * G.th, w0 = tck * TW;
             const int khv = min(G.th, G.H - h0), kwv = min(TW, G.W - w0);
             const bool full = (e & full_bit) != 0;
-            const bool need_mask = !full || khv < G.th || kwv < TW;
-            uint32_t keep[4] = {~0u, ~0u, ~0u, ~0u};
-            if (need_mask) {
-                const int s = full ? 1 << 20 : (int)my_tab[abs(tk - tq) * 128 + row];
-                int a_lo = max(0, hq - s - h0), a_hi = min(khv - 1, hq + s - h0);
-                const int b_lo = max(0, wq - s - w0), b_hi = min(kwv - 1, wq + s - w0);
-                if (!qvalid) { a_lo = 1; a_hi = 0; }
-                row_keep_bits<TWL>(a_lo, a_hi, b_lo, b_hi, keep);
+            // kept keys of this row inside the tile: key rows [a_lo, a_hi] x columns [b_lo, b_hi]
+            int a_lo = 0, a_hi = khv - 1, b_lo = 0, b_hi = kwv - 1;
+            if (!full) {
+                const int s = (int)my_tab[abs(tk - tq) * 128 + row];
+                a_lo = max(0, hq - s - h0); a_hi = min(khv - 1, hq + s - h0);
+                b_lo = max(0, wq - s - w0); b_hi = min(kwv - 1, wq + s - w0);
             }
+            if (!qvalid) { a_lo = 1; a_hi = 0; }
+            // column bias (0 kept, -inf masked) as pairs; the row bias is added per key row
+            f2_t colb[CP];
+#pragma unroll
+            for (int bp = 0; bp < CP; ++bp)
+                colb[bp] = f2_pack((2 * bp >= b_lo && 2 * bp <= b_hi) ? 0.f : -INFINITY,
+                                   (2 * bp + 1 >= b_lo && 2 * bp + 1 <= b_hi) ? 0.f : -INFINITY);
 
             const bool got = role_wait(&s_full[w], k & 1, G.wait_ns, s_abort);
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
             tc_fence_after();
             __syncwarp();
-            float s[128];
-            {
-                uint32_t v[4][32];
+            uint32_t v[4][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + c * 32, v[c]);
-                tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + c * 32, v[c]);
+            tmem_wait_ld();
+            // x = S * scale - m_run + bias  (log2 domain), packed in pairs
+            f2_t x[64];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+            for (int a = 0; a < KR; ++a) {
+                const float rb = (a >= a_lo && a <= a_hi) ? -m_run : -INFINITY;
+                const f2_t rb2 = f2_pack(rb, rb);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[c][i]);
+                for (int bp = 0; bp < CP; ++bp) {
+                    const int i = a * CP + bp, c = (2 * i) >> 5, o = (2 * i) & 31;
+                    x[i] = f2_add(f2_fma(f2_pack(__uint_as_float(v[c][o]), __uint_as_float(v[c][o + 1])), sc2, colb[bp]), rb2);
+                }
             }
-            if (need_mask) {
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 128; ++c) s[c] = (keep[c >> 5] & (1u << (c & 31))) ? s[c] : -INFINITY;
+            for (int i = 0; i < 64; ++i) {
+                float x0, x1;
+                f2_unpack(x[i], x0, x1);
+                m4[i & 3] = max3(m4[i & 3], x0, x1);
             }
-            float m4[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float a = max3(s[q * 32], s[q * 32 + 1], s[q * 32 + 2]);
-#pragma unroll
-                for (int i = 3; i < 31; i += 2) a = max3(a, s[q * 32 + i], s[q * 32 + i + 1]);
-                m4[q] = fmaxf(a, s[q * 32 + 31]);
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));   // relative to m_run
+            // shift the frame: to the first kept maximum, or up when a tile exceeds 2^8
+            float delta = 0.f, alpha = 1.f;
+            bool resc = false;
+            if (mx > -INFINITY) {
+                if (l == 0.f) delta = mx;
+                else if (mx > 8.f) { delta = mx; alpha = ex2(-mx); resc = true; }
             }
-            const float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
-            const bool need = m_tile > m_run + 8.0f;
-            float alpha = 1.f;
-            if (need) { alpha = ex2(m_run - m_tile); m_run = m_tile; }
+            if (delta != 0.f) {
+                m_run += delta;
+                const f2_t nd = f2_pack(-delta, -delta);
+#pragma unroll
+                for (int i = 0; i < 64; ++i) x[i] = f2_add(x[i], nd);
+            }
             l *= alpha;
-            const bool rescale = k > 0 && __any_sync(0xffffffffu, need);
-            const float neg_m = -m_run;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            const bool rescale = k > 0 && __any_sync(0xffffffffu, resc);
+            f2_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int e2 = c * 16 + i;                 // pair index
-                    const float x0 = fmaf(s[2 * e2], sc, neg_m);
-                    const float x1 = fmaf(s[2 * e2 + 1], sc, neg_m);
-                    pk[i] = pack_bf16x2(ex2(x0), ex2(x1));
+                for (int q = 0; q < 16; ++q) {
+                    float x0, x1;
+                    f2_unpack(x[c * 16 + q], x0, x1);
+                    pk[q] = pack_bf16x2(ex2(x0), ex2(x1));
                     // the row sum adds exactly the bf16 values the tensor core will use
-                    ls[i & 3] += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+                    ls[q & 3] = f2_add(ls[q & 3], f2_pack(__uint_as_float(pk[q] << 16), __uint_as_float(pk[q] & 0xffff0000u)));
                 }
                 tmem_st16(tmem + lane_base + colS + c * 16, pk);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            {
+                float s0, s1, s2, s3, s4, s5, s6, s7;
+                f2_unpack(ls[0], s0, s1); f2_unpack(ls[1], s2, s3); f2_unpack(ls[2], s4, s5); f2_unpack(ls[3], s6, s7);
+                l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            }
             // O_w is complete up to tile k-1 (the QK for this tile waited for that
             // PV); rescale it before PV of this tile is issued (after p_full)
             if (rescale) {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + colO + c * 32, v);
+                    uint32_t vo[32];
+                    tmem_ld32(tmem + lane_base + colO + c * 32, vo);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                    tmem_st32(tmem + lane_base + colO + c * 32, v);
+                    for (int i = 0; i < 32; ++i) vo[i] = __float_as_uint(__uint_as_float(vo[i]) * alpha);
+                    tmem_st32(tmem + lane_base + colO + c * 32, vo);
                 }
             }
             tmem_wait_st();

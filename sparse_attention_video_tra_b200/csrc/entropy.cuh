@@ -42,9 +42,9 @@ struct EntCfg {
     static constexpr int WARP_LOAD = 8, WARP_MMA = 9;     // MMA issuers: warps 9 (tile A), 10 (tile B)
 };
 
-// exp2 of the elements with (index % ENT_POLY_MOD) == ENT_POLY_MOD - 1 runs on
-// the FMA pipe (degree-4 polynomial), the rest on the MUFU unit
-constexpr int ENT_POLY_MOD = 4;
+// exp2 of the element pairs with (pair % ENT_POLY_MOD) == ENT_POLY_MOD - 1 runs
+// on the FMA pipe (degree-4 polynomial, packed pairs), the rest on the MUFU unit
+constexpr int ENT_POLY_MOD = 3;
 
 template <int D, int TWL>
 __global__ void __launch_bounds__(352, 1)
@@ -66,6 +66,7 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* drain = s_empty + 4;           // [2]
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    int* s_lock = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
 
     const int pair = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -81,6 +82,7 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(&drain[0], 1);
         mbar_init(&drain[1], 1);
         *s_abort = 0;
+        *s_lock = 0;
         fence_barrier_init();
     }
     if (warp == C::WARP_MMA) { tmem_alloc(s_tmem, 512); tmem_relinquish(); }
@@ -127,6 +129,7 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) break;
                 if (!active) { mbar_arrive(&k_empty[ks]); continue; }
                 if (j >= 2 && !role_wait(&s_empty[w * 2 + b], ((j - 2) >> 1) & 1, G.wait_ns, s_abort)) break;
+                if (!issue_lock(s_lock, G.wait_ns, s_abort)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -136,6 +139,7 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 mma_commit(&s_full[w * 2 + b]);
                 mma_commit(&k_empty[ks]);
+                issue_unlock(s_lock);
             }
             mma_commit(&drain[w]);
             mbar_wait(&drain[w], 0, G.drain_ns);
@@ -158,54 +162,57 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
             tc_fence_after();
             __syncwarp();
-            float s[128];
-            {
-                uint32_t v[4][32];
+            uint32_t v[4][32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_base + bs * 128 + q * 32, v[q]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(v[q][i]);
-            }
+            for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_base + bs * 128 + q * 32, v[q]);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_empty[bs]);
             if (edge) {                     // pad keys of edge tiles take no probability
                 uint32_t keep[4];
                 row_keep_bits<TWL>(0, khv - 1, 0, kwv - 1, keep);
 #pragma unroll
-                for (int i = 0; i < 128; ++i) s[i] = (keep[i >> 5] & (1u << (i & 31))) ? s[i] : -1e30f;
+                for (int i = 0; i < 128; ++i)
+                    if (!(keep[i >> 5] & (1u << (i & 31)))) v[i >> 5][i & 31] = __float_as_uint(-1e30f);
             }
             // four independent max chains, then combine
-            float m4[4];
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float a = max3(s[q * 32], s[q * 32 + 1], s[q * 32 + 2]);
-#pragma unroll
-                for (int i = 3; i < 31; i += 2) a = max3(a, s[q * 32 + i], s[q * 32 + i + 1]);
-                m4[q] = fmaxf(a, s[q * 32 + 31]);
-            }
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            const float mt = mx * c;
+            for (int i = 0; i < 64; ++i)
+                m4[i & 3] = max3(m4[i & 3], __uint_as_float(v[i >> 4][(2 * i) & 31]), __uint_as_float(v[i >> 4][(2 * i + 1) & 31]));
+            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
             if (mt > m) {
                 const float alpha = ex2(m - mt);
                 A = alpha * fmaf(m - mt, Z, A);
                 Z *= alpha;
                 m = mt;
             }
-            // eight independent partial sums keep the adds off one serial chain
-            float zt[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            float at[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            // u = s*c - m (<= 0), e = 2^u; Z += e, A += e*u, all in packed pairs;
+            // four independent accumulator chains
+            const f2_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
+            f2_t z2[4] = {0ull, 0ull, 0ull, 0ull}, a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                const float u = fmaf(s[i], c, -m);
-                const float e = (i % ENT_POLY_MOD == ENT_POLY_MOD - 1) ? ex2_poly<4>(u) : ex2(u);
-                zt[i & 7] += e;
-                at[i & 7] = fmaf(e, u, at[i & 7]);
+            for (int i = 0; i < 64; ++i) {
+                const f2_t u2 = f2_fma(f2_pack(__uint_as_float(v[i >> 4][(2 * i) & 31]),
+                                               __uint_as_float(v[i >> 4][(2 * i + 1) & 31])), c2, nm2);
+                f2_t e2;
+                if (i % ENT_POLY_MOD == ENT_POLY_MOD - 1) {
+                    e2 = ex2_poly4_pair(u2);
+                } else {
+                    float u0, u1;
+                    f2_unpack(u2, u0, u1);
+                    e2 = f2_pack(ex2(u0), ex2(u1));
+                }
+                z2[i & 3] = f2_add(z2[i & 3], e2);
+                a2[i & 3] = f2_fma(e2, u2, a2[i & 3]);
             }
-            Z += ((zt[0] + zt[1]) + (zt[2] + zt[3])) + ((zt[4] + zt[5]) + (zt[6] + zt[7]));
-            A += ((at[0] + at[1]) + (at[2] + at[3])) + ((at[4] + at[5]) + (at[6] + at[7]));
+            const f2_t zs = f2_add(f2_add(z2[0], z2[1]), f2_add(z2[2], z2[3]));
+            const f2_t as = f2_add(f2_add(a2[0], a2[1]), f2_add(a2[2], a2[3]));
+            float zl, zh, al, ah;
+            f2_unpack(zs, zl, zh);
+            f2_unpack(as, al, ah);
+            Z += zl + zh;
+            A += al + ah;
         }
         if (ok) {
             const float H = logf(Z) - 0.69314718055994531f * (A / Z) + corr;

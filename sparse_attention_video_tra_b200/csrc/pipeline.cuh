@@ -55,6 +55,27 @@ __device__ __forceinline__ bool poll_alive(uint64_t& t_last, bool progress, uint
     return true;
 }
 
+// A shared-memory lock that keeps the MMA groups of two issuers from
+// interleaving in the tensor pipe (an issue occupies the issuing thread about
+// as long as the MMA runs, so a group issued under the lock runs as a block).
+__device__ __forceinline__ bool issue_lock(int* lock, uint64_t limit_ns, volatile int* abort_flag)
+{
+    if (atomicCAS(lock, 0, 1) == 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        __nanosleep(20);
+        if (atomicCAS(lock, 0, 1) == 0) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicOr(&g_tra_error, TRA_ERRBIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void issue_unlock(int* lock) { atomicExch(lock, 0); }
+
 // Keep-bits of one query row inside a key tile, as four 32-column words.
 // Key (a, b) of the tile (a = key row, b = key column) is kept iff
 // a_lo <= a <= a_hi and b_lo <= b <= b_hi.

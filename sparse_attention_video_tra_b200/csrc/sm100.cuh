@@ -199,6 +199,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// Warpgroup register rebalancing (all 128 threads of the warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -257,6 +263,62 @@ __device__ __forceinline__ float ex2_poly(float x)
     }
     const float scale = __int_as_float(__float_as_int(t) << 23);   // 2^k, 0 when k = -127
     return p * scale;
+}
+
+// ---- packed fp32 pairs (sm_100 FFMA2/FADD2/FMUL2): two floats in a 64-bit register
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t f2_pack(float lo, float hi)
+{
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(f2_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c)
+{
+    f2_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+__device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b)
+{
+    f2_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b)
+{
+    f2_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 2^x for a pair, on the FMA pipe (the same method as ex2_poly<4>), for
+// x <= 0 (x <= -127 gives exactly 0).
+__device__ __forceinline__ f2_t ex2_poly4_pair(f2_t x2)
+{
+    float a, b;
+    f2_unpack(x2, a, b);
+    x2 = f2_pack(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
+    const f2_t C = f2_pack(12583039.0f, 12583039.0f);        // 1.5 * 2^23 + 127
+    const f2_t t = f2_add(x2, C);                                // round(x) in the low mantissa bits
+    const f2_t f = f2_add(x2, f2_fma(t, f2_pack(-1.0f, -1.0f), C));   // x - round(x), exact
+    f2_t p = f2_fma(f2_pack(0.0095701013f, 0.0095701013f), f, f2_pack(0.0559178591f, 0.0559178591f));
+    p = f2_fma(p, f, f2_pack(0.2402474433f, 0.2402474433f));
+    p = f2_fma(p, f, f2_pack(0.6931217909f, 0.6931217909f));
+    p = f2_fma(p, f, f2_pack(0.9999992847f, 0.9999992847f));
+    float t0, t1;
+    f2_unpack(t, t0, t1);
+    const f2_t scale = f2_pack(__int_as_float(__float_as_int(t0) << 23), __int_as_float(__float_as_int(t1) << 23));
+    return f2_mul(p, scale);
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c)

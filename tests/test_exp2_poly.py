@@ -63,3 +63,33 @@ def test_underflow_and_masked_inputs_give_zero(deg):
 def test_coefficients_parse():
     assert len(coeffs(3)) == 4 and len(coeffs(4)) == 5
     assert abs(coeffs(3)[-1] - 1) < 1e-3 and abs(coeffs(4)[-2] - np.log(2)) < 1e-3
+
+
+def pair_coeffs():
+    src = open(HDR).read()
+    body = src[src.index("ex2_poly4_pair"):]
+    body = body[:body.index("return f2_mul")]
+    vals = re.findall(r"f2_pack\((\d+\.\d+)f, \1f\)", body)
+    return [np.float32(v) for v in vals if float(v) < 1.5 and v not in ("1.0",)]
+
+
+def ex2_pair(x):
+    """The packed-pair variant: f = x + (C - t) instead of x - (t - C)."""
+    x = np.maximum(np.asarray(x, np.float32), np.float32(-127.0))
+    C = np.float32(12583039.0)
+    t = (x + C).astype(np.float32)
+    f = (x + fma32(t, np.full_like(t, np.float32(-1.0)), np.full_like(t, C))).astype(np.float32)
+    cs = pair_coeffs()
+    p = fma32(np.full_like(f, cs[0]), f, np.full_like(f, cs[1]))
+    for c in cs[2:]:
+        p = fma32(p, f, np.full_like(f, c))
+    bits = (t.view(np.int32).astype(np.int64) << 23).astype(np.uint64) & np.uint64(0xFFFFFFFF)
+    return (p * bits.astype(np.uint32).view(np.float32)).astype(np.float32)
+
+
+def test_pair_variant_matches_scalar_coefficients_and_bound():
+    assert [float(c) for c in pair_coeffs()] == [float(c) for c in coeffs(4)]
+    x = np.linspace(-120, 0, 1_000_001).astype(np.float32)
+    rel = np.abs(ex2_pair(x).astype(np.float64) / np.exp2(x.astype(np.float64)) - 1)
+    assert rel.max() <= 2.8e-6
+    assert np.all(ex2_pair(np.array([-np.inf, -1e30, -127.0], np.float32)) == 0.0)
