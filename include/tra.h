@@ -123,8 +123,9 @@ typedef struct {
  *   Bmin      smallest budget, 1 <= Bmin <= N
  *   flags     TRA_FLAG_*; 0 = defaults (tile shape with the least padding)
  * Returns TRA_ERR_INVALID_ARG for impossible values, TRA_ERR_UNSUPPORTED for
- * shapes the kernels do not handle (d not 64/128, > 32 tile columns per frame,
- * > 32767 tiles per head, r_cap >= 2^20).  No CUDA call is made.
+ * shapes the kernels do not handle (d not 64/128, H or W above 256, > 32 tile
+ * columns per frame, > 32767 tiles per head, > 2048 key tiles listed per
+ * query tile, r_cap >= 2^20).  No CUDA call is made.
  */
 TRA_API tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int heads, int d,
                            double a, double b, double gamma, int Rt, int Bmin,
