@@ -24,9 +24,11 @@
 //              while the other waits for the tensor core.
 //   warp 8     TMA producer: Q_A, Q_B, then the K and V rings.
 //   warps 9,10 MMA issuers for tiles A and B (warp 9 also allocates TMEM): for
-//              each listed key tile j, S_w = Q_w K(j)^T (once PV_w of the
-//              previous tile is complete: P_w lives in S_w), then
-//              O_w += P_w(j) V(j); the two tiles progress independently.
+//              each listed key tile j, O_w += P_w(j) V(j), and in the same issue
+//              group S_w = Q_w K(j')^T for the next listed tile j' once its K
+//              has landed (the tensor pipe runs one thread's MMAs in order, so
+//              the QK overwrites S, where P_w lives, only after the PV has read
+//              it); the two tiles progress independently.
 //   warp 11    idle (completes the third warpgroup for register rebalancing:
 //              the softmax warpgroups run with 216 registers, warps 8-11 with 72).
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
@@ -233,10 +235,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ------------------------------------------------ MMA issuers, one per query tile
         // Issuing tcgen05.mma occupies the issuing thread about as long as the
         // tensor core runs it, so each query tile w gets its own issuer; both walk
-        // the merged list in order.  For a tile w lists: S_w = Q_w K^T (once its
-        // previous PV is complete: P_w lives in S_w), then O_w += P_w V.  Either
-        // way it releases the K and V ring stages (two arrivals per occupant): a
-        // commit after its MMAs, or a plain arrive once the tile has landed.
+        // the merged list in order.  For a tile w lists: S_w = Q_w K^T, then,
+        // once the softmax has written P_w, O_w += P_w V followed in the same
+        // group by the next listed tile's QK.  Either way it releases the K and V
+        // ring stages (two arrivals per occupant): a commit after its MMAs, or a
+        // plain arrive once the tile has landed.  The softmax rescales O_w at
+        // tile k only after s_full of tile k, whose commit covers every earlier
+        // MMA of this thread, the PV of tile k-1 included.
         const int w = warp - C::WARP_MMA;
         if (lane == 0 && n > 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
@@ -245,28 +250,35 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t in_bit = MT_IN0 << w;
             bool ok = role_wait(q_full, 0, G.wait_ns, s_abort);
             int cnt = 0;
+            int qk_ahead = -1;                  // entry whose QK went out with the previous PV group
+            auto issue_qk = [&](int jj) {
+                const int kss = jj % C::KST;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
+                    mma_ss(tmem + col_s(w), smem_desc_sw128(sQa + off, 16, 1024),
+                           smem_desc_sw128(sKa + kss * C::TILE + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[w]);
+                mma_commit(&k_empty[kss]);
+            };
             for (int j = 0; ok && j < n; ++j) {
                 const bool uses = (merged[j] & in_bit) != 0;
                 const int ks = j % C::KST, vs = j % C::VST;
-                if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!uses) {
+                    if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                     mbar_arrive(&k_empty[ks]);
                     if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                     mbar_arrive(&v_empty[vs]);
                     continue;
                 }
-                if (cnt > 0 && !role_wait(&pv_done[w], (cnt - 1) & 1, G.wait_ns, s_abort)) { ok = false; break; }
-                if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
-                    mma_ss(tmem + col_s(w), smem_desc_sw128(sQa + off, 16, 1024),
-                           smem_desc_sw128(sKa + ks * C::TILE + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+                if (qk_ahead != j) {
+                    if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                    if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_qk(j);
+                    issue_unlock(s_lock);
                 }
-                mma_commit(&s_full[w]);
-                mma_commit(&k_empty[ks]);
-                issue_unlock(s_lock);
                 if (!role_wait(&p_full[w], cnt & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
@@ -278,6 +290,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                            (cnt > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&pv_done[w]);
                 mma_commit(&v_empty[vs]);
+                // The next tile's QK joins this group when this query tile lists
+                // it and its K has landed: the tensor pipe runs the MMAs of one
+                // thread in order, so the QK overwrites S (holding P) only after
+                // this PV has read P.
+                if (j + 1 < n && (merged[j + 1] & in_bit) &&
+                    mbar_test(&k_full[(j + 1) % C::KST], ((j + 1) / C::KST) & 1)) {
+                    tc_fence_after();
+                    issue_qk(j + 1);
+                    qk_ahead = j + 1;
+                }
                 issue_unlock(s_lock);
                 ++cnt;
             }
@@ -400,8 +422,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 f2_unpack(ls[0], s0, s1); f2_unpack(ls[1], s2, s3); f2_unpack(ls[2], s4, s5); f2_unpack(ls[3], s6, s7);
                 l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
             }
-            // O_w is complete up to tile k-1 (the QK for this tile waited for that
-            // PV); rescale it before PV of this tile is issued (after p_full)
+            // O_w is complete up to tile k-1 (s_full of this tile covers that PV);
+            // rescale it before the PV of this tile is issued (after p_full)
             if (rescale) {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
