@@ -377,56 +377,90 @@ def mask_algorithmic_bytes(run) -> float:
 
 
 def run_e2e(run, wl, calls, args, world):
-    """The same metric through the public API with host buffers: per step,
-    pinned host -> device copies of Q, K and each call's V (natural order),
-    tile-major permutes, the hot path, and each call's output back to host."""
-    from sparse_attention_video_tra_b200 import Plan
+    """The same metric through the public API with host buffers.  Per step:
+    pinned host -> device copies of Q, K (natural token order) and of each
+    call's V, the hot path on a natural-layout plan (TRA_FLAG_NATURAL: the
+    kernels read frame-major tensors through 4-D TMA boxes, no permute pass),
+    and each call's output back to pinned host memory.  Copies run on their
+    own streams: V of call c+1 goes up while call c computes, and the output
+    of call c comes down while call c+1 computes (V and outputs are double
+    buffered)."""
+    from sparse_attention_video_tra_b200 import Plan, TRA_FLAG_NATURAL
     i = run.info
-    plan = run.plan
+    plan = Plan(wl.T, wl.H, wl.W, wl.heads, wl.d, wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin,
+                run.plan.flags | TRA_FLAG_NATURAL)
     shape = (i.heads, i.N, i.d)
     hq = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     hk = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     hv = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
-    ho = torch.empty(shape, dtype=run.out.dtype, pin_memory=True)
+    ho = torch.empty(shape, dtype=plan.out_dtype, pin_memory=True)
     tmp = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
-    plan.permute(run.q, tmp, False); hq.copy_(tmp)
-    plan.permute(run.k, tmp, False); hk.copy_(tmp)
-    plan.permute(run.v[0], tmp, False); hv.copy_(tmp)
-    dq, dk, dv = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(3))
-    dn = torch.empty(shape, dtype=run.out.dtype, device="cuda")
+    run.plan.permute(run.q, tmp, False); hq.copy_(tmp)
+    run.plan.permute(run.k, tmp, False); hk.copy_(tmp)
+    run.plan.permute(run.v[0], tmp, False); hv.copy_(tmp)
     del tmp
+    dq, dk = plan.new_input(), plan.new_input()
+    dv = [plan.new_input(), plan.new_input()]
+    do = [plan.new_out(), plan.new_out()]
+    dH = plan.new_entropy()
+    dmask = plan.new_mask()
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()                       # noqa: E731
 
     def step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        plan.permute(dq, run.q)
-        plan.permute(dk, run.k)
-        plan.entropy(run.q, run.k, run.H, wl.key_stride)
-        plan.radius_and_mask(run.H, run.mask)
+        start = ev(); start.record(comp)
+        s_in.wait_event(start)
+        with torch.cuda.stream(s_in):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            qk_in = ev(); qk_in.record(s_in)
+        comp.wait_event(qk_in)
+        plan.entropy(dq, dk, dH, wl.key_stride, stream=comp)
+        plan.radius_and_mask(dH, dmask, stream=comp)
+        v_free = [start, start]                            # buffer b may be refilled
+        o_free = [start, start]                            # buffer b may be rewritten
+        last = start
         for c in range(calls):
-            dv.copy_(hv, non_blocking=True)
-            plan.permute(dv, run.v[c])
-            plan.attention(run.q, run.k, run.v[c], run.mask, run.out)
-            plan.permute(run.out, dn, False)
-            ho.copy_(dn, non_blocking=True)
+            b = c & 1
+            s_in.wait_event(v_free[b])
+            with torch.cuda.stream(s_in):
+                dv[b].copy_(hv, non_blocking=True)
+                v_in = ev(); v_in.record(s_in)
+            comp.wait_event(v_in)
+            comp.wait_event(o_free[b])
+            plan.attention(dq, dk, dv[b], dmask, do[b], stream=comp)
+            done = ev(); done.record(comp)
+            v_free[b] = done
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                ho.copy_(do[b], non_blocking=True)
+                out_done = ev(); out_done.record(s_out)
+            o_free[b] = out_done
+            last = out_done
+        comp.wait_event(last)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(comp)
     for _ in range(args.steps):
         step()
-    e1.record()
+    e1.record(comp)
     torch.cuda.synchronize()
     barrier(world)
+    if plan.status() != 0:
+        raise RuntimeError("device error word set during the end-to-end run")
     secs = e0.elapsed_time(e1) / 1000.0
     val = aggregate(run.attention_flops() * calls * args.steps, secs, world) / 1e12
     nbytes = i.heads * i.N * i.d * 2
-    obytes = i.heads * i.N * i.d * run.out.element_size()
+    obytes = i.heads * i.N * i.d * ho.element_size()
+    plan.close()
     return {"value": round(val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": nbytes * (2 + calls),
-            "d2h_bytes_per_step": obytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3)}
+            "d2h_bytes_per_step": obytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3),
+            "layout": "natural [heads][T][H][W][d]; copies overlapped with compute on two copy streams"}
 
 
 def main(argv=None):

@@ -87,6 +87,14 @@ typedef enum {
 #define TRA_FLAG_DEBUG_NO_WAIT (1u << 16)  /* test hook: pipeline waits give up at
                                               once, exercising the timeout path */
 #define TRA_FLAG_OUT_BF16      (1u << 17)  /* tra_attention writes bf16 instead of fp32 */
+#define TRA_FLAG_NATURAL       (1u << 18)  /* q, k, v, out and the entropies are in the
+                                              natural frame-major token order
+                                              n = (t*H + h)*W + w: [heads][N][d] and
+                                              [heads][N], no pad rows.  The kernels
+                                              load each (1, th, tw) tile straight from
+                                              it with a 4-D TMA box and store results
+                                              back to their natural rows, so no
+                                              tra_permute pass is needed. */
 
 /* everything a caller needs to size and read buffers */
 typedef struct {
@@ -158,6 +166,8 @@ TRA_API tra_status tra_permute(tra_plan plan, const void* src, void* dst, int to
  *   q, k   device bf16 [heads][N_pad][d] tile-major, 16-byte aligned; pad rows
  *          must hold finite values (tra_permute writes zeros)
  *   Hout   device fp32 [heads][N_pad]; pad rows are unspecified
+ *          (with TRA_FLAG_NATURAL: q, k bf16 [heads][N][d] and Hout fp32
+ *          [heads][N], natural token order)
  *   key_tile_stride  1 = all N keys (exact).  s > 1 = only the valid keys of
  *          key tiles whose index is a multiple of s, plus ln(N / |S|) where S
  *          is that key set (the plug-in entropy of the subsample, shifted so a
@@ -171,7 +181,8 @@ TRA_API tra_status tra_entropy(tra_plan plan, const void* q, const void* k, floa
  * tra_radius_and_mask -- budget, radius and block-sparse mask in one launch
  * ("Budget-vers-Rayon" and "Noyaux CUDA Fusionnes": distance computation,
  * radius comparison, block pruning and token voting).
- *   Hent       device fp32 [heads][N_pad] tile-major entropies (pad rows ignored)
+ *   Hent       device fp32 [heads][N_pad] tile-major entropies (pad rows ignored);
+ *              [heads][N] in natural order with TRA_FLAG_NATURAL
  *   mask       device buffer of at least mask_bytes (tra_plan_info), 256-byte
  *              aligned; layout as described in tra_plan_info.  Every field is
  *              rewritten by each call; entries past tile_count are unspecified.
@@ -193,6 +204,8 @@ TRA_API tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void* m
  *   mask       the buffer written by tra_radius_and_mask for this plan
  *   out        device [heads][N_pad][d] tile-major, fp32 (bf16 when the plan
  *              has TRA_FLAG_OUT_BF16); pad rows unspecified
+ * With TRA_FLAG_NATURAL q, k, v and out are [heads][N][d] in natural token
+ * order (the mask buffer is the same either way).
  * Asynchronous on `stream`.
  */
 TRA_API tra_status tra_attention(tra_plan plan, const void* q, const void* k, const void* v,

@@ -21,7 +21,7 @@ __all__ = [
     "TraError", "PlanInfo", "Plan", "library_path", "load_library",
     "tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
     "tra_radius_and_mask", "tra_attention", "tra_plan_status", "tra_status_string",
-    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "tra_flag_tile_w",
+    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "tra_flag_tile_w",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +31,7 @@ _lib = None
 TRA_OK = 0
 TRA_FLAG_DEBUG_NO_WAIT = 1 << 16
 TRA_FLAG_OUT_BF16 = 1 << 17
+TRA_FLAG_NATURAL = 1 << 18
 STATUS_NAMES = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARG", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_WORKSPACE",
                 4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT", 6: "TRA_ERR_DEVICE_CHECK"}
 
@@ -204,13 +205,33 @@ class Plan:
         import torch
         return torch.bfloat16 if self.flags & TRA_FLAG_OUT_BF16 else torch.float32
 
+    @property
+    def natural(self) -> bool:
+        """q, k, v, out and entropies in natural token order (TRA_FLAG_NATURAL)."""
+        return bool(self.flags & TRA_FLAG_NATURAL)
+
+    @property
+    def io_rows(self) -> int:
+        """Rows per head of q, k, v, out and the entropies in this plan's layout."""
+        return self.info.N if self.natural else self.info.N_pad
+
     def new_tile_major(self, device="cuda", dtype=None):
         import torch
         i = self.info
         return torch.empty(i.heads, i.N_pad, i.d, dtype=dtype or torch.bfloat16, device=device)
 
+    def new_input(self, device="cuda", dtype=None):
+        """A q/k/v buffer in this plan's layout."""
+        import torch
+        i = self.info
+        return torch.empty(i.heads, self.io_rows, i.d, dtype=dtype or torch.bfloat16, device=device)
+
     def new_out(self, device="cuda"):
-        return self.new_tile_major(device, self.out_dtype)
+        return self.new_input(device, self.out_dtype)
+
+    def new_entropy(self, device="cuda"):
+        import torch
+        return torch.empty(self.info.heads, self.io_rows, dtype=torch.float32, device=device)
 
     def new_mask(self, device="cuda"):
         import torch
@@ -246,26 +267,26 @@ class Plan:
     def entropy(self, q, k, Hout, key_tile_stride=1, stream=None):
         import torch
         i = self.info
-        self._rows(q, i.N_pad, "q")
-        self._rows(k, i.N_pad, "k")
-        if Hout.dtype != torch.float32 or not Hout.is_cuda or Hout.numel() != i.heads * i.N_pad:
-            raise ValueError("Hout: expected cuda float32 [heads, N_pad]")
+        self._rows(q, self.io_rows, "q")
+        self._rows(k, self.io_rows, "k")
+        if Hout.dtype != torch.float32 or not Hout.is_cuda or Hout.numel() != i.heads * self.io_rows:
+            raise ValueError(f"Hout: expected cuda float32 [heads, {self.io_rows}]")
         tra_entropy(self.handle, q.data_ptr(), k.data_ptr(), Hout.data_ptr(), key_tile_stride, self._stream(stream))
         return Hout
 
     def radius_and_mask(self, Hent, mask, stream=None):
         import torch
         i = self.info
-        if Hent.dtype != torch.float32 or not Hent.is_cuda or Hent.numel() != i.heads * i.N_pad:
-            raise ValueError("Hent: expected cuda float32 [heads, N_pad]")
+        if Hent.dtype != torch.float32 or not Hent.is_cuda or Hent.numel() != i.heads * self.io_rows:
+            raise ValueError(f"Hent: expected cuda float32 [heads, {self.io_rows}]")
         tra_radius_and_mask(self.handle, Hent.data_ptr(), mask.data_ptr(), mask.numel(), self._stream(stream))
         return mask
 
     def attention(self, q, k, v, mask, out, stream=None):
         i = self.info
         for x, nme in ((q, "q"), (k, "k"), (v, "v")):
-            self._rows(x, i.N_pad, nme)
-        self._rows(out, i.N_pad, "out", self.out_dtype)
+            self._rows(x, self.io_rows, nme)
+        self._rows(out, self.io_rows, "out", self.out_dtype)
         tra_attention(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), mask.data_ptr(), out.data_ptr(),
                       self._stream(stream))
         return out

@@ -193,9 +193,6 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t* sK = smem + C::OFF_K;
     uint8_t* sV = smem + C::OFF_V;
     const int kbase = g * G.N_pad;
-    auto key_row = [&](uint32_t e) {
-        return kbase + (((int)(e & 0x7fff) * G.nTh + (int)((e >> 15) & 63)) * G.nTw + (int)((e >> 21) & 31)) * 128;
-    };
 
     if (warp >= C::WARP_LOAD) {
       regs_dec<C::REGS_OTHER>();
@@ -204,26 +201,30 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0 && n > 0) {
             prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
+            int tqa, trqa, tcqa, tqb, trqb, tcqb;
+            tile_coords(G, qa, tqa, trqa, tcqa);
+            tile_coords(G, hasB ? qb : qa, tqb, trqb, tcqb);
 #pragma unroll
             for (int p = 0; p < C::NP; ++p) {
-                tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, kbase + qa * 128, q_full);
-                if (hasB) tma_load_2d(sQ + C::TILE + p * C::PANEL, &tm_q, p * 64, kbase + qb * 128, q_full);
+                load_tile_panel(sQ + p * C::PANEL, &tm_q, G, p, g, tqa, trqa, tcqa, q_full);
+                if (hasB) load_tile_panel(sQ + C::TILE + p * C::PANEL, &tm_q, G, p, g, tqb, trqb, tcqb, q_full);
             }
             int kiss = 0, viss = 0;
             for (int j = 0; j < n; ++j) {
-                const int y = key_row(merged[j]);
+                const uint32_t e = merged[j];
+                const int tk = (int)(e & 0x7fff), trk = (int)((e >> 15) & 63), tck = (int)((e >> 21) & 31);
                 const int ks = j % C::KST, vs = j % C::VST;
                 if (j >= C::KST && !role_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, G.wait_ns, s_abort)) break;
                 mbar_arrive_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
                 for (int p = 0; p < C::NP; ++p)
-                    tma_load_2d(sK + ks * C::TILE + p * C::PANEL, &tm_k, p * 64, y, &k_full[ks]);
+                    load_tile_panel(sK + ks * C::TILE + p * C::PANEL, &tm_k, G, p, g, tk, trk, tck, &k_full[ks]);
                 ++kiss;
                 if (j >= C::VST && !role_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, G.wait_ns, s_abort)) break;
                 mbar_arrive_expect_tx(&v_full[vs], C::TILE);
 #pragma unroll
                 for (int p = 0; p < C::NP; ++p)
-                    tma_load_2d(sV + vs * C::TILE + p * C::PANEL, &tm_v, p * 64, y, &v_full[vs]);
+                    load_tile_panel(sV + vs * C::TILE + p * C::PANEL, &tm_v, G, p, g, tk, trk, tck, &v_full[vs]);
                 ++viss;
             }
             // copies still in flight must land before the CTA exits
@@ -446,12 +447,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tc_fence_after();
                 __syncwarp();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                const size_t orow = (size_t)(kbase + qt * 128 + row) * D;
+                const bool store = !G.natural || qvalid;          // natural layout has no pad rows
+                const size_t orow = io_row(G, g, tq, hq, wq, qt * 128 + row) * D;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(tmem + lane_base + colO + c * 32, v);
                     tmem_wait_ld();
+                    if (!store) continue;
                     if constexpr (OUT_BF16) {
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + orow + c * 32);
                         uint32_t o[16];

@@ -73,7 +73,6 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int qa = 2 * pair, qb = 2 * pair + 1;
     const bool hasB = qb < G.nQ;
     const int n = (G.nQ + stride - 1) / stride;              // key tiles visited
-    const int kbase = g * G.N_pad;
 
     if (tid == 0) {
         mbar_init(q_full, 1);
@@ -94,19 +93,24 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (lane == 0) {
             prefetch_tmap(&tm_q); prefetch_tmap(&tm_k);
             mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
+            int ta, tra_, tca, tb, trb, tcb;
+            tile_coords(G, qa, ta, tra_, tca);
+            tile_coords(G, hasB ? qb : qa, tb, trb, tcb);
 #pragma unroll
             for (int p = 0; p < C::NP; ++p) {
-                tma_load_2d(sQ + p * C::PANEL, &tm_q, p * 64, kbase + qa * 128, q_full);
-                if (hasB) tma_load_2d(sQ + C::TILE + p * C::PANEL, &tm_q, p * 64, kbase + qb * 128, q_full);
+                load_tile_panel(sQ + p * C::PANEL, &tm_q, G, p, g, ta, tra_, tca, q_full);
+                if (hasB) load_tile_panel(sQ + C::TILE + p * C::PANEL, &tm_q, G, p, g, tb, trb, tcb, q_full);
             }
             int issued = 0;
             for (int j = 0; j < n; ++j) {
                 const int st = j % C::KST;
                 if (j >= C::KST && !role_wait(&k_empty[st], ((j / C::KST) - 1) & 1, G.wait_ns, s_abort)) break;
                 mbar_arrive_expect_tx(&k_full[st], C::TILE);
+                int tk, trk, tck;
+                tile_coords(G, j * stride, tk, trk, tck);
 #pragma unroll
                 for (int p = 0; p < C::NP; ++p)
-                    tma_load_2d(sK + st * C::TILE + p * C::PANEL, &tm_k, p * 64, kbase + j * stride * 128, &k_full[st]);
+                    load_tile_panel(sK + st * C::TILE + p * C::PANEL, &tm_k, G, p, g, tk, trk, tck, &k_full[st]);
                 ++issued;
             }
             mbar_wait(q_full, 0, G.drain_ns);
@@ -216,7 +220,11 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         if (ok) {
             const float H = logf(Z) - 0.69314718055994531f * (A / Z) + corr;
-            Hout[kbase + (w ? qb : qa) * 128 + row] = H;
+            const int qt = w ? qb : qa;
+            int tq, trq, tcq;
+            tile_coords(G, qt, tq, trq, tcq);
+            const int hq = trq * G.th + (row >> TWL), wq = tcq * TW + (row & (TW - 1));
+            if (!G.natural || (hq < G.H && wq < G.W)) Hout[io_row(G, g, tq, hq, wq, qt * 128 + row)] = H;
         }
     }
     tc_fence_before();

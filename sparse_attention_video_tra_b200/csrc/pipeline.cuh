@@ -76,6 +76,20 @@ __device__ __forceinline__ bool issue_lock(int* lock, uint64_t limit_ns, volatil
 
 __device__ __forceinline__ void issue_unlock(int* lock) { atomicExch(lock, 0); }
 
+// One 64-column panel of a 128-row tile (frame t, tile row tr, tile column
+// tc, head g) into shared memory.  Tile-major inputs: rows tile*128 ..
+// tile*128+127 of a [rows][d] map.  Natural inputs: a {64, tw, th, 1} box of a
+// [heads*T][H][W][d] map, which lands in the same row order (row = (h - h0)*tw
+// + (w - w0)); positions past the grid's edge read as zeros.
+__device__ __forceinline__ void load_tile_panel(void* dst, const CUtensorMap* m, const Geom& G, int p, int g, int t,
+                                                int tr, int tc, uint64_t* bar)
+{
+    if (G.natural)
+        tma_load_4d(dst, m, p * 64, tc * G.tw, tr * G.th, g * G.T + t, bar);
+    else
+        tma_load_2d(dst, m, p * 64, g * G.N_pad + ((t * G.nTh + tr) * G.nTw + tc) * 128, bar);
+}
+
 // Keep-bits of one query row inside a key tile, as four 32-column words.
 // Key (a, b) of the tile (a = key row, b = key column) is kept iff
 // a_lo <= a <= a_hi and b_lo <= b <= b_hi.

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     int r = -1;
     long long c = 0;
     if (valid) {
-        const long long bh = budget_hat(G, Hent[row]);
+        const long long bh = budget_hat(G, Hent[io_row(G, g, t, h, w, tile * 128 + tid)]);
         int lo = 0, hi = G.r_cap;
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;

@@ -51,6 +51,27 @@ bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, int D)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [heads*T][H][W][D] bf16 in natural token order, {64, tw, th, 1} boxes (one
+// panel of one (1, th, tw) tile; coordinates past the grid read as zeros)
+bool make_natural_map(CUtensorMap* m, const void* base, const tra::Geom& G)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)G.D, (cuuint64_t)G.W, (cuuint64_t)G.H, (cuuint64_t)G.T * G.G};
+    const cuuint64_t strides[3] = {(cuuint64_t)G.D * 2, (cuuint64_t)G.W * G.D * 2, (cuuint64_t)G.H * G.W * G.D * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)G.tw, (cuuint32_t)G.th, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// the input map for the plan's layout
+bool make_input_map(CUtensorMap* m, const void* base, const tra::Geom& G)
+{
+    return G.natural ? make_natural_map(m, base, G) : make_row_map(m, base, (uint64_t)G.G * G.N_pad, G.D);
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 tra_status launch_status()
@@ -125,8 +146,7 @@ extern "C" tra_status tra_entropy(tra_plan plan, const void* q, const void* k, f
         corr = (float)std::log((double)G.N / (double)nS);
     }
     CUtensorMap mq, mk;
-    const uint64_t rows = (uint64_t)G.G * G.N_pad;
-    if (!make_row_map(&mq, q, rows, G.D) || !make_row_map(&mk, k, rows, G.D)) return TRA_ERR_CUDA;
+    if (!make_input_map(&mq, q, G) || !make_input_map(&mk, k, G)) return TRA_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     const int key = G.D * 100 + G.tw_log2;
     switch (key) {
@@ -160,8 +180,7 @@ extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k,
         return TRA_ERR_INVALID_ARG;
     const tra::Geom& G = plan->geom;
     CUtensorMap mq, mk, mv;
-    const uint64_t rows = (uint64_t)G.G * G.N_pad;
-    if (!make_row_map(&mq, q, rows, G.D) || !make_row_map(&mk, k, rows, G.D) || !make_row_map(&mv, v, rows, G.D))
+    if (!make_input_map(&mq, q, G) || !make_input_map(&mk, k, G) || !make_input_map(&mv, v, G))
         return TRA_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     const uint8_t* m = (const uint8_t*)mask;

@@ -26,4 +26,11 @@ __device__ __forceinline__ void tile_coords(const Geom& G, int tile, int& t, int
     tc = rem - tr * G.nTw;
 }
 
+// Row of token (t, h, w) of head g in the caller's layout: natural order, or
+// row `tile_row` (tile*128 + in-tile row) of the tile-major layout.
+__device__ __forceinline__ size_t io_row(const Geom& G, int g, int t, int h, int w, int tile_row)
+{
+    return G.natural ? (size_t)g * G.N + ((size_t)t * G.H + h) * G.W + w : (size_t)g * G.N_pad + tile_row;
+}
+
 }  // namespace tra

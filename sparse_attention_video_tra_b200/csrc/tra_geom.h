@@ -27,6 +27,7 @@ struct Geom {
     float scale_log2;                // log2(e) / sqrt(d)
     unsigned long long wait_ns;      // limit of a pipeline wait
     unsigned long long drain_ns;     // limit of the waits that drain in-flight copies
+    int natural;                     // q/k/v/out/entropies in natural token order (4-D TMA boxes)
 };
 
 }  // namespace tra

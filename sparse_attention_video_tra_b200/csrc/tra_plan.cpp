@@ -47,7 +47,8 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     const long long N = (long long)T * H * W;
     if (Bmin < 1 || (long long)Bmin > N) return TRA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return TRA_ERR_UNSUPPORTED;
-    if (flags & ~(TRA_FLAG_TILE_W_MASK | TRA_FLAG_DEBUG_NO_WAIT | TRA_FLAG_OUT_BF16)) return TRA_ERR_INVALID_ARG;
+    if (flags & ~(TRA_FLAG_TILE_W_MASK | TRA_FLAG_DEBUG_NO_WAIT | TRA_FLAG_OUT_BF16 | TRA_FLAG_NATURAL))
+        return TRA_ERR_INVALID_ARG;
 
     if (H > TRA_MAX_HW || W > TRA_MAX_HW) return TRA_ERR_UNSUPPORTED;
     const int rte = Rt < T - 1 ? Rt : T - 1;
@@ -109,6 +110,7 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     G.a = a; G.b = b; G.Bmin = Bmin;
     G.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     G.wait_ns = (flags & TRA_FLAG_DEBUG_NO_WAIT) ? 0ull : 2000000000ull;
+    G.natural = (flags & TRA_FLAG_NATURAL) ? 1 : 0;
     G.drain_ns = 2000000000ull;
 
     // mask buffer layout

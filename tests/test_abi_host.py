@@ -67,6 +67,18 @@ def test_plan_create_rejects(args, status):
     assert e.value.status == status
 
 
+def test_natural_layout_flag():
+    """TRA_FLAG_NATURAL: q/k/v/out/entropies hold N rows per head in natural
+    token order; unknown flag bits are still rejected."""
+    p = tra.Plan(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=tra.TRA_FLAG_NATURAL)
+    assert p.natural and p.io_rows == p.info.N == 256
+    q = tra.Plan(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8)
+    assert not q.natural and q.io_rows == q.info.N_pad
+    assert p.info == q.info                      # same geometry and mask layout
+    with pytest.raises(tra.TraError):
+        tra.tra_plan_create(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=1 << 19)
+
+
 def test_plan_create_rejects_bad_flags():
     with pytest.raises(tra.TraError) as e:
         tra.tra_plan_create(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=1 << 3)
