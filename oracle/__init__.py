@@ -55,24 +55,25 @@ def lib() -> ctypes.CDLL:
         L.oracle_halfwidth.restype = ctypes.c_int64
         L.oracle_rt_eff.argtypes = [ctypes.c_int, ctypes.c_int]
         L.oracle_rt_eff.restype = ctypes.c_int
-        L.oracle_r_cap.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        L.oracle_r_cap.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
         L.oracle_r_cap.restype = ctypes.c_int64
-        L.oracle_count.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int] + [ctypes.c_int] * 3 + [ctypes.c_int64]
+        L.oracle_count.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int] + [ctypes.c_int] * 3 + \
+            [ctypes.c_int64, ctypes.c_int]
         L.oracle_count.restype = ctypes.c_int64
         L.oracle_budget.argtypes = [ctypes.c_float, ctypes.c_double, ctypes.c_double, ctypes.c_int64, ctypes.c_int64]
         L.oracle_budget.restype = ctypes.c_int64
         L.oracle_radius.argtypes = [_F32P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_int,
-                                    _I64P, ctypes.c_int64, _I32P, _I64P, _I64P]
-        L.oracle_token_mask.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int,
+                                    ctypes.c_int, _I64P, ctypes.c_int64, _I32P, _I64P, _I64P]
+        L.oracle_token_mask.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                                              ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
         L.oracle_token_mask.restype = ctypes.c_int
-        L.oracle_block_mask.argtypes = [_I32P] + [ctypes.c_int] * 4 + [ctypes.c_double, ctypes.c_int] + \
+        L.oracle_block_mask.argtypes = [_I32P] + [ctypes.c_int] * 4 + [ctypes.c_double, ctypes.c_int, ctypes.c_int] + \
             [ctypes.c_int] * 4 + [_I64P, ctypes.c_int64, _U8P]
         L.oracle_entropy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 5 + \
             [ctypes.c_int] * 3 + [_I64P, ctypes.c_int64, _F64P]
         L.oracle_attention.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, _I32P] + [ctypes.c_int] * 5 + \
-            [ctypes.c_double, ctypes.c_int, _I64P, ctypes.c_int64, _F64P]
+            [ctypes.c_double, ctypes.c_int, ctypes.c_int, _I64P, ctypes.c_int64, _F64P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -116,24 +117,28 @@ def rt_eff(T: int, Rt: int) -> int:
     return int(lib().oracle_rt_eff(T, Rt))
 
 
-def r_cap(T: int, H: int, W: int, gamma: float, Rt: int) -> int:
-    return int(lib().oracle_r_cap(T, H, W, gamma, Rt))
+# metric: 0 = Chebyshev square (the default reading), 1 = Euclidean disk
+CHEBYSHEV, DISK = 0, 1
 
 
-def count(T, H, W, gamma, Rt, t, h, w, r) -> int:
-    return int(lib().oracle_count(T, H, W, gamma, Rt, t, h, w, r))
+def r_cap(T: int, H: int, W: int, gamma: float, Rt: int, metric: int = CHEBYSHEV) -> int:
+    return int(lib().oracle_r_cap(T, H, W, gamma, Rt, metric))
+
+
+def count(T, H, W, gamma, Rt, t, h, w, r, metric: int = CHEBYSHEV) -> int:
+    return int(lib().oracle_count(T, H, W, gamma, Rt, t, h, w, r, metric))
 
 
 def budget(Hent: float, a: float, b: float, N: int, Bmin: int) -> int:
     return int(lib().oracle_budget(float(np.float32(Hent)), a, b, N, Bmin))
 
 
-def token_mask(T, H, W, gamma, Rt, i, j, r_i) -> bool:
-    return bool(lib().oracle_token_mask(T, H, W, gamma, Rt, i, j, r_i))
+def token_mask(T, H, W, gamma, Rt, i, j, r_i, metric: int = CHEBYSHEV) -> bool:
+    return bool(lib().oracle_token_mask(T, H, W, gamma, Rt, metric, i, j, r_i))
 
 
 # ----------------------------------------------------------------- arrays
-def radius(Hent, G, grid, a, b, gamma, Rt, Bmin, queries=None):
+def radius(Hent, G, grid, a, b, gamma, Rt, Bmin, queries=None, metric: int = CHEBYSHEV):
     """E3+E4.  Hent: fp32 entropies (all G*N in order, or one per listed query).
     Returns (r int32, c int64, bhat int64) per row."""
     T, H, W = grid
@@ -144,12 +149,12 @@ def radius(Hent, G, grid, a, b, gamma, Rt, Bmin, queries=None):
     r = np.zeros(rows, np.int32)
     c = np.zeros(rows, np.int64)
     bh = np.zeros(rows, np.int64)
-    lib().oracle_radius(_ptr(Hf, _F32P), G, T, H, W, a, b, gamma, Rt, Bmin,
+    lib().oracle_radius(_ptr(Hf, _F32P), G, T, H, W, a, b, gamma, Rt, Bmin, metric,
                         qp, nq, _ptr(r, _I32P), _ptr(c, _I64P), _ptr(bh, _I64P))
     return r, c, bh
 
 
-def block_mask(r, G, grid, gamma, Rt, qtile, ktile, qtiles=None) -> np.ndarray:
+def block_mask(r, G, grid, gamma, Rt, qtile, ktile, qtiles=None, metric: int = CHEBYSHEV) -> np.ndarray:
     """E6.  r: int32 radii [G*N] natural order.  qtile/ktile: (th, tw) of the
     (1, th, tw) query/key tiles.  Returns uint8 [rows, nK]: 0 inactive,
     1 active, 3 active and full.  qtiles: list of g*nQ + a (None = all)."""
@@ -162,7 +167,7 @@ def block_mask(r, G, grid, gamma, Rt, qtile, ktile, qtiles=None) -> np.ndarray:
     q, nq, qp = _qlist(qtiles)
     rows = nq if q is not None else G * nQ
     out = np.zeros((rows, nK), np.uint8)
-    lib().oracle_block_mask(_ptr(rr, _I32P), G, T, H, W, gamma, Rt, qth, qtw, kth, ktw,
+    lib().oracle_block_mask(_ptr(rr, _I32P), G, T, H, W, gamma, Rt, metric, qth, qtw, kth, ktw,
                             qp, nq, _ptr(out, _U8P))
     return out
 
@@ -181,7 +186,7 @@ def entropy(q, k, G, grid, d, key_stride=1, ktile=(1, 1), queries=None) -> np.nd
     return out
 
 
-def attention(q, k, v, r, G, grid, d, gamma, Rt, queries=None) -> np.ndarray:
+def attention(q, k, v, r, G, grid, d, gamma, Rt, queries=None, metric: int = CHEBYSHEV) -> np.ndarray:
     """E7: masked softmax attention, fp64 [rows, d]."""
     T, H, W = grid
     qa, tq = _elems(q)
@@ -193,7 +198,7 @@ def attention(q, k, v, r, G, grid, d, gamma, Rt, queries=None) -> np.ndarray:
     rows = nq if ql is not None else G * T * H * W
     out = np.zeros((rows, d), np.float64)
     lib().oracle_attention(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, tq, _ptr(rr, _I32P),
-                           G, T, H, W, d, gamma, Rt, qp, nq, _ptr(out, _F64P))
+                           G, T, H, W, d, gamma, Rt, metric, qp, nq, _ptr(out, _F64P))
     return out
 
 

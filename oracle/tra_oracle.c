@@ -32,7 +32,11 @@
  *   - counts are taken over in-grid keys only;
  *   - "token voting" is an OR vote: a tile pair is active iff any retained
  *     token pair lies in it;
- *   - subsampled entropy: plug-in entropy over the sampled keys + ln(N/|S|).
+ *   - subsampled entropy: plug-in entropy over the sampled keys + ln(N/|S|);
+ *   - metric 1 (the summary's "circular neighbourhoods" / 2D disk mask): the
+ *     spatial test is dh^2 + dw^2 <= s^2 with the same half-width s; the
+ *     count then sums, row by row, the clipped width 2*isqrt(s^2 - dh^2) + 1,
+ *     and r_cap is the smallest r with s(r, Rt')^2 >= (H-1)^2 + (W-1)^2.
  *
  * Build:  gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
  * (fp-contract=off keeps r*g and +1e-9 as two separately rounded operations).
@@ -105,20 +109,41 @@ int oracle_rt_eff(int T, int Rt) { return Rt < T - 1 ? Rt : T - 1; }
 
 /* r_cap: the smallest r whose farthest-frame half-width reaches the grid,
    s(r, Rt') >= max(H, W) - 1, so no larger radius adds keys. */
-int64_t oracle_r_cap(int T, int H, int W, double gamma, int Rt)
+int64_t oracle_r_cap(int T, int H, int W, double gamma, int Rt, int metric)
 {
     int rte = oracle_rt_eff(T, Rt);
     double g = pow(gamma, (double)rte);
-    int64_t need = (H > W ? H : W) - 1;
     int64_t r = 0;
+    if (metric == 1) {
+        /* the farthest-frame disk must reach the opposite corner of the frame */
+        int64_t need2 = (int64_t)(H - 1) * (H - 1) + (int64_t)(W - 1) * (W - 1);
+        for (;;) {
+            int64_t s = oracle_halfwidth(r, g);
+            if (s * s >= need2) return r;
+            ++r;
+        }
+    }
+    int64_t need = (H > W ? H : W) - 1;
     while (oracle_halfwidth(r, g) < need) ++r;
     return r;
+}
+
+/* the largest integer x >= 0 with x*x <= n (n >= 0), by bisection */
+static int64_t isqrt_floor(int64_t n)
+{
+    int64_t lo = 0, hi = 1;
+    while (hi * hi <= n) hi *= 2;
+    while (hi - lo > 1) {
+        int64_t mid = (lo + hi) / 2;
+        if (mid * mid <= n) lo = mid; else hi = mid;
+    }
+    return lo;
 }
 
 /* c_i(r): number of in-grid keys j with |t_i-t_j| <= Rt' and Chebyshev
    distance <= s(r, |t_i - t_j|), by the clipped-rectangle formula. */
 int64_t oracle_count(int T, int H, int W, double gamma, int Rt,
-                     int t, int h, int w, int64_t r)
+                     int t, int h, int w, int64_t r, int metric)
 {
     int rte = oracle_rt_eff(T, Rt);
     int64_t c = 0;
@@ -127,8 +152,17 @@ int64_t oracle_count(int T, int H, int W, double gamma, int Rt,
         if (tt < 0 || tt >= T) continue;
         int64_t s = oracle_halfwidth(r, pow(gamma, (double)(dt < 0 ? -dt : dt)));
         int64_t hl = imax64(0, h - s), hh = imin64(H - 1, h + s);
-        int64_t wl = imax64(0, w - s), wh = imin64(W - 1, w + s);
-        c += (hh - hl + 1) * (wh - wl + 1);
+        if (metric == 1) {
+            /* disk: each key row h' holds the keys with dw^2 <= s^2 - dh^2 */
+            for (int64_t hk = hl; hk <= hh; ++hk) {
+                int64_t dh = hk - h;
+                int64_t half = isqrt_floor(s * s - dh * dh);
+                c += imin64(W - 1, w + half) - imax64(0, w - half) + 1;
+            }
+        } else {
+            int64_t wl = imax64(0, w - s), wh = imin64(W - 1, w + s);
+            c += (hh - hl + 1) * (wh - wl + 1);
+        }
     }
     return c;
 }
@@ -150,13 +184,13 @@ int64_t oracle_budget(float Hent, double a, double b, int64_t N, int64_t Bmin)
    r_i = the smallest r in [0, r_cap] with c_i(r) >= Bhat_i, found by a
    linear scan upward from 0 (the definition), else r_cap. */
 void oracle_radius(const float* Hent, int G, int T, int H, int W,
-                   double a, double b, double gamma, int Rt, int Bmin,
+                   double a, double b, double gamma, int Rt, int Bmin, int metric,
                    const int64_t* queries, int64_t n_queries,
                    int32_t* r_out, int64_t* c_out, int64_t* bhat_out)
 {
     grid_t gr = {T, H, W};
     int64_t N = (int64_t)T * H * W;
-    int64_t rcap = oracle_r_cap(T, H, W, gamma, Rt);
+    int64_t rcap = oracle_r_cap(T, H, W, gamma, Rt, metric);
     int64_t rows = queries ? n_queries : (int64_t)G * N;
     #pragma omp parallel for schedule(dynamic, 64)
     for (int64_t row = 0; row < rows; ++row) {
@@ -164,10 +198,10 @@ void oracle_radius(const float* Hent, int G, int T, int H, int W,
         int t, h, w;
         coords(&gr, gi % N, &t, &h, &w);
         int64_t bh = oracle_budget(Hent[row], a, b, N, Bmin);
-        int64_t r = 0, c = oracle_count(T, H, W, gamma, Rt, t, h, w, 0);
+        int64_t r = 0, c = oracle_count(T, H, W, gamma, Rt, t, h, w, 0, metric);
         while (c < bh && r < rcap) {
             ++r;
-            c = oracle_count(T, H, W, gamma, Rt, t, h, w, r);
+            c = oracle_count(T, H, W, gamma, Rt, t, h, w, r, metric);
         }
         r_out[row] = (int32_t)r;
         if (c_out) c_out[row] = c;
@@ -176,7 +210,7 @@ void oracle_radius(const float* Hent, int G, int T, int H, int W,
 }
 
 /* E5: token mask M_ij given the query's radius ([TRA] "Budget-vers-Rayon") */
-static int token_mask(const grid_t* gr, double gamma, int rte,
+static int token_mask(const grid_t* gr, double gamma, int rte, int metric,
                       int64_t i, int64_t j, int64_t r_i)
 {
     int ti, hi, wi, tj, hj, wj;
@@ -187,15 +221,16 @@ static int token_mask(const grid_t* gr, double gamma, int rte,
     int64_t s = oracle_halfwidth(r_i, pow(gamma, (double)dt));
     int64_t dh = hi > hj ? hi - hj : hj - hi;
     int64_t dw = wi > wj ? wi - wj : wj - wi;
+    if (metric == 1) return dh * dh + dw * dw <= s * s;    /* disk */
     int64_t cheb = dh > dw ? dh : dw;
     return cheb <= s;
 }
 
-int oracle_token_mask(int T, int H, int W, double gamma, int Rt,
+int oracle_token_mask(int T, int H, int W, double gamma, int Rt, int metric,
                       int64_t i, int64_t j, int64_t r_i)
 {
     grid_t gr = {T, H, W};
-    return token_mask(&gr, gamma, oracle_rt_eff(T, Rt), i, j, r_i);
+    return token_mask(&gr, gamma, oracle_rt_eff(T, Rt), metric, i, j, r_i);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -209,7 +244,7 @@ int oracle_token_mask(int T, int H, int W, double gamma, int Rt,
 /* retained pair), 3 active and full (every valid pair retained).            */
 /* ------------------------------------------------------------------------ */
 void oracle_block_mask(const int32_t* r, int G, int T, int H, int W,
-                       double gamma, int Rt,
+                       double gamma, int Rt, int metric,
                        int qth, int qtw, int kth, int ktw,
                        const int64_t* qtiles, int64_t n_qtiles,
                        uint8_t* out)
@@ -240,7 +275,7 @@ void oracle_block_mask(const int32_t* r, int G, int T, int H, int W,
                     int hj = bh * kth + jh, wj = bw * ktw + jw;
                     if (hj >= H || wj >= W) continue;
                     int64_t j = ((int64_t)bt * H + hj) * W + wj;
-                    if (token_mask(&gr, gamma, rte, i, j, r[g * N + i])) any = 1;
+                    if (token_mask(&gr, gamma, rte, metric, i, j, r[g * N + i])) any = 1;
                     else all = 0;
                 }
             }
@@ -317,7 +352,7 @@ void oracle_entropy(const void* q, const void* k, int type,
 /* ------------------------------------------------------------------------ */
 void oracle_attention(const void* q, const void* k, const void* v, int type,
                       const int32_t* r, int G, int T, int H, int W, int d,
-                      double gamma, int Rt,
+                      double gamma, int Rt, int metric,
                       const int64_t* queries, int64_t n_queries, double* out)
 {
     grid_t gr = {T, H, W};
@@ -335,7 +370,7 @@ void oracle_attention(const void* q, const void* k, const void* v, int type,
             int64_t g = gi / N, i = gi % N;
             double m = -INFINITY;
             for (int64_t j = 0; j < N; ++j) {
-                if (!token_mask(&gr, gamma, rte, i, j, r[gi])) { s[j] = -INFINITY; continue; }
+                if (!token_mask(&gr, gamma, rte, metric, i, j, r[gi])) { s[j] = -INFINITY; continue; }
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c)
                     acc += load_elem(q, (size_t)gi * d + c, type)

@@ -30,16 +30,20 @@ def halfwidth(r, g):
     return np.floor(prod + 1e-9).astype(np.int64)
 
 
-def token_mask(T, H, W, gamma, Rt, r):
-    """Dense boolean M[i, j] for radii r[i] (natural order)."""
+def token_mask(T, H, W, gamma, Rt, r, disk=False):
+    """Dense boolean M[i, j] for radii r[i] (natural order).  disk=True takes
+    the Euclidean test dh^2 + dw^2 <= s^2 instead of the Chebyshev one."""
     t, h, w = coords(T, H, W)
     rte = min(Rt, T - 1)
     g = decay(gamma, rte)
     dt = np.abs(t[:, None] - t[None, :])
-    cheb = np.maximum(np.abs(h[:, None] - h[None, :]), np.abs(w[:, None] - w[None, :]))
+    dh = np.abs(h[:, None] - h[None, :])
+    dw = np.abs(w[:, None] - w[None, :])
     inside = dt <= rte
     s = halfwidth(np.asarray(r)[:, None], g[np.minimum(dt, rte)])
-    return inside & (cheb <= s)
+    if disk:
+        return inside & (dh * dh + dw * dw <= s * s)
+    return inside & (np.maximum(dh, dw) <= s)
 
 
 def bhat(Hent, a, b, N, Bmin):
@@ -51,26 +55,32 @@ def bhat(Hent, a, b, N, Bmin):
     return np.array(out, dtype=np.int64)
 
 
-def r_cap(T, H, W, gamma, Rt):
+def r_cap(T, H, W, gamma, Rt, disk=False):
+    """Smallest r at which no query's mask row can grow any more: the
+    farthest-frame test reaches the whole frame from every position."""
     rte = min(Rt, T - 1)
     g = decay(gamma, rte)[rte]
-    need = max(H, W) - 1
     r = 0
+    if disk:
+        while int(halfwidth(r, g)) ** 2 < (H - 1) ** 2 + (W - 1) ** 2:
+            r += 1
+        return r
+    need = max(H, W) - 1
     while int(halfwidth(r, g)) < need:
         r += 1
     return r
 
 
-def radius(Hent, T, H, W, a, b, gamma, Rt, Bmin):
+def radius(Hent, T, H, W, a, b, gamma, Rt, Bmin, disk=False):
     """Smallest r whose dense token-mask row holds >= Bhat keys, else r_cap.
     Returns (r, counts) for one head (Hent of length N)."""
     N = T * H * W
     bh = bhat(Hent, a, b, N, Bmin)
-    rc = r_cap(T, H, W, gamma, Rt)
+    rc = r_cap(T, H, W, gamma, Rt, disk)
     r = np.full(N, -1, dtype=np.int64)
     cnt = np.zeros(N, dtype=np.int64)
     for rr in range(rc + 1):
-        c = token_mask(T, H, W, gamma, Rt, np.full(N, rr)).sum(axis=1)
+        c = token_mask(T, H, W, gamma, Rt, np.full(N, rr), disk).sum(axis=1)
         newly = (r < 0) & (c >= bh)
         r[newly] = rr
         cnt[newly] = c[newly]
