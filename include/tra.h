@@ -95,6 +95,13 @@ typedef enum {
                                               it with a 4-D TMA box and store results
                                               back to their natural rows, so no
                                               tra_permute pass is needed. */
+#define TRA_FLAG_DISK          (1u << 19)  /* Euclidean-disk spatial test
+                                              dh^2 + dw^2 <= s^2 (the summary's
+                                              circular neighbourhoods) instead of
+                                              the Chebyshev square max(|dh|,|dw|)
+                                              <= s; same half-width s.  r_cap is
+                                              then the smallest r with
+                                              s(r, Rt')^2 >= (H-1)^2 + (W-1)^2. */
 
 /* everything a caller needs to size and read buffers */
 typedef struct {

@@ -21,7 +21,7 @@ __all__ = [
     "TraError", "PlanInfo", "Plan", "library_path", "load_library",
     "tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
     "tra_radius_and_mask", "tra_attention", "tra_plan_status", "tra_status_string",
-    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "tra_flag_tile_w",
+    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "TRA_FLAG_DISK", "tra_flag_tile_w",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,6 +32,7 @@ TRA_OK = 0
 TRA_FLAG_DEBUG_NO_WAIT = 1 << 16
 TRA_FLAG_OUT_BF16 = 1 << 17
 TRA_FLAG_NATURAL = 1 << 18
+TRA_FLAG_DISK = 1 << 19
 STATUS_NAMES = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARG", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_WORKSPACE",
                 4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT", 6: "TRA_ERR_DEVICE_CHECK"}
 

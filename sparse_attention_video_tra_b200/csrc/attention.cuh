@@ -69,8 +69,8 @@ struct AttnDyn {
         // key tiles a pair of query tiles can reach: frames t-Rt' .. t+1+Rt'
         L.bw = ((2 * rte + 2) * tiles_per_frame + 31) / 32;
         L.merged = 0;                                               // uint32 [2 * list_cap]
-        L.stab = L.merged + 8 * list_cap;                           // uint8 [2][rte + 1][128]
-        L.bits = L.stab + ((2 * (rte + 1) * 128 + 15) & ~15);       // uint32 [5][bw]
+        L.stab = L.merged + 8 * list_cap;                           // uint16 [2][rte + 1][128]
+        L.bits = L.stab + ((2 * (rte + 1) * 128 * 2 + 15) & ~15);   // uint32 [5][bw]
         L.bars = L.bits + ((5 * L.bw * 4 + 15) & ~15);              // uint64 [32]
         L.misc = L.bars + 8 * 32;
         L.total = L.misc + 16;
@@ -92,7 +92,7 @@ __device__ __forceinline__ uint32_t pack_tile(int t, int tr, int tc)
 }
 constexpr uint32_t MT_IN0 = 1u << 26, MT_FULL0 = 1u << 28;
 
-template <int D, int TWL, bool OUT_BF16>
+template <int D, int TWL, bool OUT_BF16, bool DISK>
 __global__ void __launch_bounds__(384, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Geom G, const uint8_t* __restrict__ mask,
@@ -105,7 +105,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const AttnDyn L = AttnDyn::make(G.list_cap, G.rte, G.tiles_per_frame);
     uint8_t* dyn = smem + C::OFF_DYN;
     uint32_t* merged = reinterpret_cast<uint32_t*>(dyn + L.merged);
-    uint8_t* s_tab = dyn + L.stab;
+    uint16_t* s_tab = reinterpret_cast<uint16_t*>(dyn + L.stab);
     uint32_t* bits = reinterpret_cast<uint32_t*>(dyn + L.bits);      // [5][bw]
     uint64_t* bars = reinterpret_cast<uint64_t*>(dyn + L.bars);
     uint64_t* q_full = bars;
@@ -324,9 +324,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int wq = tcq * TW + (row & (TW - 1));
         const bool qvalid = active && hq < G.H && wq < G.W;
         const int rq = qvalid ? reinterpret_cast<const int32_t*>(mask + G.off_radius)[kbase + qt * 128 + row] : -1;
-        uint8_t* my_tab = s_tab + w * (G.rte + 1) * 128;
+        uint16_t* my_tab = s_tab + w * (G.rte + 1) * 128;
         for (int dl = 0; dl <= G.rte; ++dl)
-            my_tab[dl * 128 + row] = (uint8_t)(qvalid ? min(halfwidth(rq, G.g[dl]), 255) : 0);
+            my_tab[dl * 128 + row] = (uint16_t)(qvalid ? min(halfwidth(rq, G.g[dl]), TRA_DISK_S_CLAMP) : 0);
         const float sc = G.scale_log2;
         const uint32_t in_bit = MT_IN0 << w, full_bit = MT_FULL0 << w;
 
@@ -348,8 +348,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const bool full = (e & full_bit) != 0;
             // kept keys of this row inside the tile: key rows [a_lo, a_hi] x columns [b_lo, b_hi]
             int a_lo = 0, a_hi = khv - 1, b_lo = 0, b_hi = kwv - 1;
+            const int s = full ? 0 : (int)my_tab[abs(tk - tq) * 128 + row];
             if (!full) {
-                const int s = (int)my_tab[abs(tk - tq) * 128 + row];
                 a_lo = max(0, hq - s - h0); a_hi = min(khv - 1, hq + s - h0);
                 b_lo = max(0, wq - s - w0); b_hi = min(kwv - 1, wq + s - w0);
             }
@@ -375,10 +375,29 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int a = 0; a < KR; ++a) {
                 const float rb = (a >= a_lo && a <= a_hi) ? -m_run : -INFINITY;
                 const f2_t rb2 = f2_pack(rb, rb);
+                if constexpr (DISK) {
+                    // the disk keeps, on key row a, the columns within
+                    // isqrt(s^2 - dh^2) of the query column
+                    int blo = b_lo, bhi = b_hi;
+                    if (!full) {
+                        const int dh = h0 + a - hq;
+                        const int half = dh * dh <= s * s ? isqrt_floor(s * s - dh * dh) : -1;
+                        blo = max(0, wq - half - w0);
+                        bhi = min(kwv - 1, wq + half - w0);
+                    }
 #pragma unroll
-                for (int bp = 0; bp < CP; ++bp) {
-                    const int i = a * CP + bp, c = (2 * i) >> 5, o = (2 * i) & 31;
-                    x[i] = f2_add(f2_fma(f2_pack(__uint_as_float(v[c][o]), __uint_as_float(v[c][o + 1])), sc2, colb[bp]), rb2);
+                    for (int bp = 0; bp < CP; ++bp) {
+                        const int i = a * CP + bp, c = (2 * i) >> 5, o = (2 * i) & 31;
+                        const f2_t cb = f2_pack((2 * bp >= blo && 2 * bp <= bhi) ? 0.f : -INFINITY,
+                                                (2 * bp + 1 >= blo && 2 * bp + 1 <= bhi) ? 0.f : -INFINITY);
+                        x[i] = f2_add(f2_fma(f2_pack(__uint_as_float(v[c][o]), __uint_as_float(v[c][o + 1])), sc2, cb), rb2);
+                    }
+                } else {
+#pragma unroll
+                    for (int bp = 0; bp < CP; ++bp) {
+                        const int i = a * CP + bp, c = (2 * i) >> 5, o = (2 * i) & 31;
+                        x[i] = f2_add(f2_fma(f2_pack(__uint_as_float(v[c][o]), __uint_as_float(v[c][o + 1])), sc2, colb[bp]), rb2);
+                    }
                 }
             }
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};

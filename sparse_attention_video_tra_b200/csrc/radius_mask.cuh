@@ -25,7 +25,9 @@
 
 namespace tra {
 
-// clipped neighbourhood count c(r) of the query at (t, h, w)
+// clipped neighbourhood count c(r) of the query at (t, h, w): per frame the
+// Chebyshev square is a clipped rectangle; the disk sums, key row by key row,
+// the clipped width 2*isqrt(s^2 - dh^2) + 1
 __device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int w, int r)
 {
     long long c = 0;
@@ -33,9 +35,21 @@ __device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int 
         const int m = (t + dl < G.T ? 1 : 0) + (dl > 0 && t - dl >= 0 ? 1 : 0);
         if (m == 0) break;                         // farther frames are out of the grid too
         const int s = halfwidth(r, G.g[dl]);
-        const int X = min(h, s) + min(G.H - 1 - h, s) + 1;
-        const int Y = min(w, s) + min(G.W - 1 - w, s) + 1;
-        c += (long long)(m * X) * Y;
+        if (G.disk) {
+            const int sc = min(s, TRA_DISK_S_CLAMP);
+            const int hl = max(0, h - sc), hh = min(G.H - 1, h + sc);
+            long long X = 0;
+            for (int hk = hl; hk <= hh; ++hk) {
+                const int dh = hk - h;
+                const int half = isqrt_floor(sc * sc - dh * dh);
+                X += min(G.W - 1, w + half) - max(0, w - half) + 1;
+            }
+            c += m * X;
+        } else {
+            const int X = min(h, s) + min(G.H - 1 - h, s) + 1;
+            const int Y = min(w, s) + min(G.W - 1 - w, s) + 1;
+            c += (long long)(m * X) * Y;
+        }
     }
     return c;
 }
@@ -54,6 +68,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     __shared__ int s_lo[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];
     __shared__ int s_hi[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];
     __shared__ int s_full[TRA_MAX_RT_EFF + 1][4];
+    __shared__ uint32_t s_fullbits[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];   // disk: full tile columns per row
     __shared__ int s_len[TRA_MAX_LIST_ROWS];
     __shared__ long long s_pairs[4];
     __shared__ int s_warp[4];
@@ -70,6 +85,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     for (int i = tid; i < (G.rte + 1) * TRA_MAX_TILES_H; i += 128) {
         (&s_lo[0][0])[i] = 0x7fffffff;
         (&s_hi[0][0])[i] = -1;
+        (&s_fullbits[0][0])[i] = 0xffffffffu;
     }
     if (tid < G.rte + 1) {
         s_full[tid][0] = -0x7fffffff; s_full[tid][1] = 0x7fffffff;
@@ -128,8 +144,18 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         const int r_hi = __reduce_max_sync(0xffffffffu, rh);
         for (int tr = r_lo; tr <= r_hi; ++tr) {
             const bool in = rl <= tr && tr <= rh;
-            const int lo = __reduce_min_sync(0xffffffffu, in ? cl : 0x7fffffff);
-            const int hi = __reduce_max_sync(0xffffffffu, in ? ch : -1);
+            int c_lo = cl, c_hi = ch;
+            if (G.disk && in) {
+                // the disk is widest on the tile row's key row nearest to h
+                const int s = min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP);
+                const int k0 = tr * G.th, k1 = min(G.H - 1, k0 + G.th - 1);
+                const int dh = h < k0 ? k0 - h : (h > k1 ? h - k1 : 0);
+                const int half = isqrt_floor(s * s - dh * dh);
+                c_lo = max(0, w - half) >> G.tw_log2;
+                c_hi = min(G.W - 1, w + half) >> G.tw_log2;
+            }
+            const int lo = __reduce_min_sync(0xffffffffu, in ? c_lo : 0x7fffffff);
+            const int hi = __reduce_max_sync(0xffffffffu, in ? c_hi : -1);
             if (lane == 0 && hi >= 0) {
                 atomicMin(&s_lo[dl][tr], lo);
                 atomicMax(&s_hi[dl][tr], hi);
@@ -137,6 +163,30 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         }
     }
     __syncthreads();
+
+    // ---- disk: a listed tile is full iff, for every valid query, its valid
+    // key rectangle's farthest corner lies in the disk (the disk is convex)
+    if (G.disk) {
+        for (int dl = 0; dl <= G.rte; ++dl) {
+            if (!(t + dl < G.T || t - dl >= 0)) break;
+            const int s = valid ? min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP) : 0;
+            for (int tr = 0; tr < G.nTh; ++tr) {
+                const int lo = s_lo[dl][tr], hi = s_hi[dl][tr];
+                if (hi < 0) continue;
+                const int k0 = tr * G.th, k1 = min(G.H - 1, k0 + G.th - 1);
+                const int dh = max(abs(h - k0), abs(h - k1));
+                uint32_t bits = 0;
+                for (int tc = lo; tc <= hi; ++tc) {
+                    const int j0 = tc * G.tw, j1 = min(G.W - 1, j0 + G.tw - 1);
+                    const int dw = max(abs(w - j0), abs(w - j1));
+                    const bool in = !valid || (long long)dh * dh + (long long)dw * dw <= (long long)s * s;
+                    if (__all_sync(0xffffffffu, in)) bits |= 1u << tc;
+                }
+                if (lane == 0) atomicAnd(&s_fullbits[dl][tr], bits | ~(((2u << hi) - 1u) ^ ((1u << lo) - 1u)));
+            }
+        }
+        __syncthreads();
+    }
 
     // ---- list rows (frame, tile row) in ascending tile order; block prefix sum
     const int t0 = max(0, t - G.rte), t1 = min(G.T - 1, t + G.rte);
@@ -166,9 +216,11 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         const int dl = abs(t0 + f - t);
         const int lo = s_lo[dl][tr], hi = s_hi[dl][tr];
         const bool row_full = s_full[dl][0] <= tr && tr <= s_full[dl][1];
+        const uint32_t fbits = s_fullbits[dl][tr];
         const int base = ((t0 + f) * G.nTh + tr) * G.nTw;
         for (int tc = lo; tc <= hi; ++tc) {
-            const bool full = row_full && s_full[dl][2] <= tc && tc <= s_full[dl][3];
+            const bool full = G.disk ? ((fbits >> tc) & 1u) != 0
+                                     : (row_full && s_full[dl][2] <= tc && tc <= s_full[dl][3]);
             list[off++] = (uint16_t)((base + tc) | (full ? 0x8000 : 0));
         }
     }

@@ -88,12 +88,12 @@ bool set_smem(K kernel, int bytes)
 // largest dynamic shared memory a CTA may use on sm_100
 constexpr int kMaxSmem = 232448;
 
-template <int D, int TWL, bool OB>
+template <int D, int TWL, bool OB, bool DISK>
 tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                          const uint8_t* mask, void* out, cudaStream_t st)
 {
     using C = tra::AttnCfg<D>;
-    auto kern = tra::attention_kernel<D, TWL, OB>;
+    auto kern = tra::attention_kernel<D, TWL, OB, DISK>;
     const int smem = tra::attn_smem_bytes<D>(G.list_cap, G.rte, G.tiles_per_frame);
     if (smem > kMaxSmem) return TRA_ERR_UNSUPPORTED;
     if (!set_smem(kern, smem)) return TRA_ERR_CUDA;
@@ -172,6 +172,37 @@ extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void
     return launch_status();
 }
 
+namespace {
+
+template <int D, int TWL>
+tra_status attention_variant(const tra::Geom& G, bool ob, bool disk, const CUtensorMap& q, const CUtensorMap& k,
+                             const CUtensorMap& v, const uint8_t* m, void* out, cudaStream_t st)
+{
+    if (ob) return disk ? run_attention<D, TWL, true, true>(G, q, k, v, m, out, st)
+                        : run_attention<D, TWL, true, false>(G, q, k, v, m, out, st);
+    return disk ? run_attention<D, TWL, false, true>(G, q, k, v, m, out, st)
+                : run_attention<D, TWL, false, false>(G, q, k, v, m, out, st);
+}
+
+// kernel instance by (head dim, tile width, output type, spatial metric)
+tra_status dispatch_attention(const tra::Geom& G, bool ob, bool disk, const CUtensorMap& q, const CUtensorMap& k,
+                              const CUtensorMap& v, const uint8_t* m, void* out, cudaStream_t st)
+{
+    switch (G.D * 100 + G.tw_log2) {
+        case 6402: return attention_variant<64, 2>(G, ob, disk, q, k, v, m, out, st);
+        case 6403: return attention_variant<64, 3>(G, ob, disk, q, k, v, m, out, st);
+        case 6404: return attention_variant<64, 4>(G, ob, disk, q, k, v, m, out, st);
+        case 6405: return attention_variant<64, 5>(G, ob, disk, q, k, v, m, out, st);
+        case 12802: return attention_variant<128, 2>(G, ob, disk, q, k, v, m, out, st);
+        case 12803: return attention_variant<128, 3>(G, ob, disk, q, k, v, m, out, st);
+        case 12804: return attention_variant<128, 4>(G, ob, disk, q, k, v, m, out, st);
+        case 12805: return attention_variant<128, 5>(G, ob, disk, q, k, v, m, out, st);
+    }
+    return TRA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
 extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k, const void* v, const void* mask,
                                     void* out, tra_stream stream)
 {
@@ -184,26 +215,9 @@ extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k,
         return TRA_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     const uint8_t* m = (const uint8_t*)mask;
-    const int key = G.D * 100 + G.tw_log2 + ((plan->flags & TRA_FLAG_OUT_BF16) ? 10 : 0);
-    switch (key) {
-        case 6402: return run_attention<64, 2, false>(G, mq, mk, mv, m, out, st);
-        case 6403: return run_attention<64, 3, false>(G, mq, mk, mv, m, out, st);
-        case 6404: return run_attention<64, 4, false>(G, mq, mk, mv, m, out, st);
-        case 6405: return run_attention<64, 5, false>(G, mq, mk, mv, m, out, st);
-        case 12802: return run_attention<128, 2, false>(G, mq, mk, mv, m, out, st);
-        case 12803: return run_attention<128, 3, false>(G, mq, mk, mv, m, out, st);
-        case 12804: return run_attention<128, 4, false>(G, mq, mk, mv, m, out, st);
-        case 12805: return run_attention<128, 5, false>(G, mq, mk, mv, m, out, st);
-        case 6412: return run_attention<64, 2, true>(G, mq, mk, mv, m, out, st);
-        case 6413: return run_attention<64, 3, true>(G, mq, mk, mv, m, out, st);
-        case 6414: return run_attention<64, 4, true>(G, mq, mk, mv, m, out, st);
-        case 6415: return run_attention<64, 5, true>(G, mq, mk, mv, m, out, st);
-        case 12812: return run_attention<128, 2, true>(G, mq, mk, mv, m, out, st);
-        case 12813: return run_attention<128, 3, true>(G, mq, mk, mv, m, out, st);
-        case 12814: return run_attention<128, 4, true>(G, mq, mk, mv, m, out, st);
-        case 12815: return run_attention<128, 5, true>(G, mq, mk, mv, m, out, st);
-    }
-    return TRA_ERR_UNSUPPORTED;
+    const bool ob = (plan->flags & TRA_FLAG_OUT_BF16) != 0;
+    const bool disk = G.disk != 0;
+    return dispatch_attention(G, ob, disk, mq, mk, mv, m, out, st);
 }
 
 extern "C" tra_status tra_plan_status(tra_plan plan)

@@ -28,6 +28,7 @@ struct Geom {
     unsigned long long wait_ns;      // limit of a pipeline wait
     unsigned long long drain_ns;     // limit of the waits that drain in-flight copies
     int natural;                     // q/k/v/out/entropies in natural token order (4-D TMA boxes)
+    int disk;                        // spatial test dh^2 + dw^2 <= s^2 instead of the Chebyshev square
 };
 
 }  // namespace tra

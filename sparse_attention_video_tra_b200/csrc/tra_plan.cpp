@@ -47,7 +47,8 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     const long long N = (long long)T * H * W;
     if (Bmin < 1 || (long long)Bmin > N) return TRA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return TRA_ERR_UNSUPPORTED;
-    if (flags & ~(TRA_FLAG_TILE_W_MASK | TRA_FLAG_DEBUG_NO_WAIT | TRA_FLAG_OUT_BF16 | TRA_FLAG_NATURAL))
+    if (flags & ~(TRA_FLAG_TILE_W_MASK | TRA_FLAG_DEBUG_NO_WAIT | TRA_FLAG_OUT_BF16 | TRA_FLAG_NATURAL |
+                  TRA_FLAG_DISK))
         return TRA_ERR_INVALID_ARG;
 
     if (H > TRA_MAX_HW || W > TRA_MAX_HW) return TRA_ERR_UNSUPPORTED;
@@ -94,8 +95,16 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     if (G.list_cap > TRA_MAX_LIST_CAP) return TRA_ERR_UNSUPPORTED;
     for (int k = 0; k <= rte; ++k) G.g[k] = std::pow(gamma, (double)k);
 
-    // r_cap: smallest r with s(r, Rt') >= max(H, W) - 1
-    const long long need = (H > W ? H : W) - 1;
+    // r_cap: the smallest r whose farthest-frame half-width s(r, Rt') reaches
+    // every key of a frame from every query: s >= max(H, W) - 1 for the
+    // Chebyshev square, s >= ceil(sqrt((H-1)^2 + (W-1)^2)) for the disk
+    const bool disk = (flags & TRA_FLAG_DISK) != 0;
+    long long need = (H > W ? H : W) - 1;
+    if (disk) {
+        const long long d2 = (long long)(H - 1) * (H - 1) + (long long)(W - 1) * (W - 1);
+        need = 0;
+        while (need * need < d2) ++need;
+    }
     const double gl = G.g[rte];
     if ((double)need / gl > (double)TRA_MAX_R_CAP) return TRA_ERR_UNSUPPORTED;
     long long r = (long long)((double)need / gl) - 2;
@@ -106,6 +115,7 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
         if (r >= TRA_MAX_R_CAP) return TRA_ERR_UNSUPPORTED;
     }
     G.r_cap = (int)r;
+    G.disk = disk ? 1 : 0;
 
     G.a = a; G.b = b; G.Bmin = Bmin;
     G.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));

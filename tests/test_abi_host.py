@@ -76,7 +76,19 @@ def test_natural_layout_flag():
     assert not q.natural and q.io_rows == q.info.N_pad
     assert p.info == q.info                      # same geometry and mask layout
     with pytest.raises(tra.TraError):
-        tra.tra_plan_create(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=1 << 19)
+        tra.tra_plan_create(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=1 << 20)
+
+
+@pytest.mark.parametrize("grid,gamma,Rt", [((21, 45, 80), 0.8, 6), ((4, 8, 8), 0.7, 2), ((3, 7, 9), 0.5, 1),
+                                           ((132, 45, 80), 0.7, 16), ((2, 256, 256), 0.9, 1)])
+def test_disk_flag_r_cap_matches_oracle(grid, gamma, Rt):
+    """TRA_FLAG_DISK: r_cap is the smallest r whose farthest-frame disk reaches
+    the opposite frame corner, as the oracle's metric-1 definition."""
+    T, H, W = grid
+    p = tra.Plan(T, H, W, 1, 128, 1.0, 0.0, gamma, Rt, 8, flags=tra.TRA_FLAG_DISK)
+    assert p.info.r_cap == oracle.r_cap(T, H, W, gamma, Rt, oracle.DISK)
+    q = tra.Plan(T, H, W, 1, 128, 1.0, 0.0, gamma, Rt, 8)
+    assert p.info.r_cap >= q.info.r_cap
 
 
 def test_plan_create_rejects_bad_flags():
