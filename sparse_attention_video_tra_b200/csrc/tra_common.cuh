@@ -17,18 +17,19 @@ __device__ __forceinline__ int halfwidth(int r, double g)
     return (int)floor(s);
 }
 
-// the largest x >= 0 with x*x <= n, for 0 <= n < 2^31
+// a half-width at which the disk already covers any frame of at most
+// TRA_MAX_HW x TRA_MAX_HW keys (keeps s*s below 2^20)
+constexpr int TRA_DISK_S_CLAMP = 1023;
+
+// the largest x >= 0 with x*x <= n, for 0 <= n <= 1023^2.  n is exact in
+// fp32 and sqrtf rounds correctly; with k = that x, sqrt(n) lies in
+// [k, k + 1 - 1/(2(k+1))] and 1/(2(k+1)) >= 2^-11 exceeds half an fp32 ulp
+// at k + 1 <= 1024 (2^-14), so the rounded root never reaches k + 1 and its
+// floor is k.
 __device__ __forceinline__ int isqrt_floor(int n)
 {
-    int x = (int)sqrtf((float)n);
-    while (x > 0 && (long long)x * x > n) --x;
-    while ((long long)(x + 1) * (x + 1) <= n) ++x;
-    return x;
+    return (int)sqrtf((float)n);
 }
-
-// a half-width at which the disk already covers any frame of at most
-// TRA_MAX_HW x TRA_MAX_HW keys (keeps s*s in 32 bits)
-constexpr int TRA_DISK_S_CLAMP = 1023;
 
 // tile index -> (frame, tile row, tile col)
 __device__ __forceinline__ void tile_coords(const Geom& G, int tile, int& t, int& tr, int& tc)
