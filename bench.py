@@ -75,9 +75,19 @@ def barrier(world: int):
         dist.barrier()
 
 
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def aggregate(per_rank_units: float, per_rank_seconds: float, world: int) -> float:
     """Whole-job throughput: units of all ranks over the slowest rank's time."""
-    return per_rank_units * world / max_over_ranks(per_rank_seconds, world)
+    return sum_over_ranks(per_rank_units, world) / max_over_ranks(per_rank_seconds, world)
 
 
 # ---------------------------------------------------------------- clocks
@@ -273,6 +283,15 @@ def run_tra(args, rank, world):
         import dataclasses
         wl = dataclasses.replace(wl, heads=args.heads, name=wl.name.replace(f"{wl.heads} heads", f"{args.heads} heads"))
     calls = args.calls if args.calls else (10 if args.workload == "wan720" else 1)
+    total_heads, workload_name = wl.heads, wl.name
+    if args.shard == "heads":
+        # strong scaling: this rank's contiguous slice of the heads
+        import dataclasses
+        from sparse_attention_video_tra_b200.runner import shard_heads
+        first, count = shard_heads(wl.heads, world, rank)
+        if count == 0:
+            raise SystemExit(f"rank {rank}: no heads left to shard ({wl.heads} heads over {world} ranks)")
+        wl = dataclasses.replace(wl, heads=count)
     run = WorkloadRun(wl, calls=calls, seed_offset=rank)
     dev_idx = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
@@ -354,12 +373,17 @@ def run_tra(args, rank, world):
     e2e = None if args.no_e2e else run_e2e(run, wl, calls, args, world)
     b_used, retained = run.b, run.retained_fraction_now()
     del run
+    sharded = args.shard == "heads"
     line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
+            "dtype": "bf16",
             "data": "synthetic (seeded Q,K,V with Wan-720p attention shapes; no model weights)",
-            "config": {"workload": wl.name, "global_batch": wl.heads * world, "seq_len": wl.N,
-                       "parallelism": f"independent head-batch replicas x{world}", "attention_calls_per_step": calls,
+            "config": {"workload": workload_name,
+                       "global_batch": total_heads if sharded else wl.heads * world, "seq_len": wl.N,
+                       "parallelism": (f"heads sharded over {world} GPUs, no collective on the path" if sharded
+                                       else f"independent head-batch replicas x{world}"),
+                       "attention_calls_per_step": calls,
                        "a": wl.a, "b": round(b_used, 6), "gamma": wl.gamma, "Rt": wl.Rt, "Bmin": wl.Bmin,
                        "inputs": "resident in HBM, 774 MB per tensor (> L2); L2 flushed before every step"},
             "retained_fraction": round(retained, 5), "phases": phases, "step_tflops": round(step_tflops, 3),
@@ -472,6 +496,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan720")
     ap.add_argument("--calls", type=int, default=0)
     ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
+    ap.add_argument("--shard", default="replica", choices=["replica", "heads"],
+                    help="replica: every rank runs the whole workload (weak scaling); "
+                         "heads: the workload's heads are split over the ranks (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -14,6 +14,19 @@ import torch
 from . import Plan, synth
 
 
+def shard_heads(heads: int, world: int, rank: int) -> tuple[int, int]:
+    """Heads of one rank when a workload's heads are split over `world` GPUs:
+    (first head, count).  Contiguous, disjoint, covering all heads, sizes
+    differing by at most one.  Heads are independent attention problems, so
+    no collective is needed on the path."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank outside the world")
+    base, extra = divmod(int(heads), int(world))
+    count = base + (1 if rank < extra else 0)
+    first = rank * base + min(rank, extra)
+    return first, count
+
+
 class WorkloadRun:
     """One workload on one GPU.
 

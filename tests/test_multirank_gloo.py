@@ -35,7 +35,9 @@ def _worker(rank, world, port, out):
         m = bench.max_over_ranks(float(rank + 1) * 1.5, world)
         # weak scaling: every rank did the same units; the slowest time divides
         agg = bench.aggregate(100.0, 1.0 + rank, world)
-        out.put((rank, m, agg))
+        # head sharding: unequal units per rank are summed, the slowest time divides
+        agg_sharded = bench.aggregate(10.0 * (rank + 1), 2.0, world)
+        out.put((rank, m, agg, agg_sharded))
         bench.barrier(world)
     finally:
         dist.destroy_process_group()
@@ -52,9 +54,10 @@ def test_two_rank_timing_and_aggregate():
         p.join(timeout=120)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(2))
-    for rank, m, agg in res:
+    for rank, m, agg, agg_sharded in res:
         assert m == 3.0                     # the max over ranks reaches every rank
         assert agg == pytest.approx(100.0 * 2 / 2.0)
+        assert agg_sharded == pytest.approx((10.0 + 20.0) / 2.0)
 
 
 def test_single_rank_is_identity():
@@ -62,3 +65,22 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(2.5, 1) == 2.5
     assert bench.aggregate(10.0, 2.0, 1) == 5.0
+
+
+@pytest.mark.parametrize("heads,world", [(40, 1), (40, 2), (40, 3), (40, 8), (24, 5), (7, 8)])
+def test_shard_heads_partitions_the_heads(heads, world):
+    """Head sharding (the path splits by head with no exchange step): the
+    ranks' slices are contiguous, disjoint, cover every head and differ in
+    size by at most one."""
+    sys.path.insert(0, ROOT)
+    from sparse_attention_video_tra_b200.runner import shard_heads
+    seen = []
+    sizes = []
+    for r in range(world):
+        first, count = shard_heads(heads, world, r)
+        seen.extend(range(first, first + count))
+        sizes.append(count)
+    assert seen == list(range(heads))
+    assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        shard_heads(heads, world, world)
