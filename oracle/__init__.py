@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             [ctypes.c_int] * 3 + [_I64P, ctypes.c_int64, _F64P]
         L.oracle_attention.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, _I32P] + [ctypes.c_int] * 5 + \
             [ctypes.c_double, ctypes.c_int, ctypes.c_int, _I64P, ctypes.c_int64, _F64P]
+        L.oracle_topk_count.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 5 + \
+            [ctypes.c_double, _I64P, ctypes.c_int64, _I64P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -199,6 +201,21 @@ def attention(q, k, v, r, G, grid, d, gamma, Rt, queries=None, metric: int = CHE
     out = np.zeros((rows, d), np.float64)
     lib().oracle_attention(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, tq, _ptr(rr, _I32P),
                            G, T, H, W, d, gamma, Rt, metric, qp, nq, _ptr(out, _F64P))
+    return out
+
+
+def topk_count(q, k, G, grid, d, mass, queries=None) -> np.ndarray:
+    """Calibration: per query, the fewest highest-probability keys whose dense
+    softmax probabilities sum to at least `mass` (exact fp64 sort)."""
+    T, H, W = grid
+    qa, tq = _elems(q)
+    ka, tk = _elems(k)
+    assert tq == tk
+    ql, nq, qp = _qlist(queries)
+    rows = nq if ql is not None else G * T * H * W
+    out = np.zeros(rows, np.int64)
+    lib().oracle_topk_count(qa.ctypes.data, ka.ctypes.data, tq, G, T, H, W, d, float(mass), qp, nq,
+                            _ptr(out, _I64P))
     return out
 
 

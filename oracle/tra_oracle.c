@@ -394,6 +394,57 @@ void oracle_attention(const void* q, const void* k, const void* v, int type,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Calibration ([TRA] Intuition I: the key density a query needs follows its */
+/* entropy): k_i(mass) = the smallest k whose k largest dense softmax       */
+/* probabilities sum to at least mass, by an exact sort of the fp64          */
+/* probabilities.  queries: NULL = all G*N, else G*N-indexed list.           */
+/* ------------------------------------------------------------------------ */
+static int cmp_desc(const void* a, const void* b)
+{
+    double x = *(const double*)a, y = *(const double*)b;
+    return x < y ? 1 : (x > y ? -1 : 0);
+}
+
+void oracle_topk_count(const void* q, const void* k, int type, int G, int T, int H, int W, int d,
+                       double mass, const int64_t* queries, int64_t n_queries, int64_t* k_out)
+{
+    int64_t N = (int64_t)T * H * W;
+    double sigma = 1.0 / sqrt((double)d);
+    int64_t rows = queries ? n_queries : (int64_t)G * N;
+    (void)G;
+    #pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)N);
+        #pragma omp for schedule(dynamic, 16)
+        for (int64_t row = 0; row < rows; ++row) {
+            int64_t gi = queries ? queries[row] : row;
+            int64_t g = gi / N;
+            double m = -INFINITY;
+            for (int64_t j = 0; j < N; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c)
+                    acc += load_elem(q, (size_t)gi * d + c, type)
+                         * load_elem(k, ((size_t)(g * N + j)) * d + c, type);
+                p[j] = acc * sigma;
+                if (p[j] > m) m = p[j];
+            }
+            double Z = 0.0;
+            for (int64_t j = 0; j < N; ++j) { p[j] = exp(p[j] - m); Z += p[j]; }
+            for (int64_t j = 0; j < N; ++j) p[j] /= Z;
+            qsort(p, (size_t)N, sizeof(double), cmp_desc);
+            double cum = 0.0;
+            int64_t kk = N;
+            for (int64_t j = 0; j < N; ++j) {
+                cum += p[j];
+                if (cum >= mass) { kk = j + 1; break; }
+            }
+            k_out[row] = kk;
+        }
+        free(p);
+    }
+}
+
 /* threads the OpenMP runtime will use (for the reported CPU baseline) */
 int oracle_num_threads(void)
 {

@@ -132,3 +132,15 @@ def block_mask(M, T, H, W, qtile, ktile):
             if blk.any():
                 out[a, b] = 3 if blk.all() else 1
     return out
+
+
+def topk_count(q, k, mass):
+    """Fewest top keys whose dense softmax probabilities reach `mass`, per row
+    (numpy sort, one head)."""
+    d = q.shape[-1]
+    s = (q.astype(np.float64) @ k.astype(np.float64).T) / math.sqrt(d)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    c = np.cumsum(-np.sort(-p, axis=1), axis=1)
+    return (c < mass).sum(axis=1) + 1
