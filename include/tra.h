@@ -219,6 +219,29 @@ TRA_API tra_status tra_attention(tra_plan plan, const void* q, const void* k, co
                          const void* mask, void* out, tra_stream stream);
 
 /*
+ * tra_calibrate_topk -- calibration workload (the summary's Intuition I: the
+ * key density a query needs follows its entropy, B ~ tau * exp(H_i)).  For the
+ * queries of every s-th query tile it returns the dense entropy H_i (computed
+ * as tra_entropy with stride 1, bit for bit) and k_i, the fewest of the
+ * query's highest-probability keys whose probabilities sum to at least
+ * `mass`.  A log-linear fit ln k = a*H + b over the returned pairs gives the
+ * plan's (a, b).  k_i is found by bisection on a log2-domain score threshold
+ * (33 passes over all keys, scores recomputed on the tensor cores); with
+ * near-equal probabilities at the cut it may differ from an exact sort by the
+ * keys whose fp32 and exact scores order differently.
+ *   q, k    bf16 queries and keys in the plan's layout (as tra_entropy)
+ *   mass    0 < mass < 1
+ *   query_tile_stride  s >= 1; n_sample = ceil(n_tiles / s) tiles per head
+ *   H_out   device fp32 [heads][n_sample][128]: tile-major rows of each
+ *           sampled tile (sampled tile i is tile i*s); NaN on pad rows
+ *   k_out   device int32 [heads][n_sample][128]; -1 on pad rows
+ * Returns TRA_ERR_INVALID_ARG for a mass outside (0, 1) or s < 1.
+ * Asynchronous on `stream`.
+ */
+TRA_API tra_status tra_calibrate_topk(tra_plan plan, const void* q, const void* k, double mass,
+                                      int query_tile_stride, float* H_out, int* k_out, tra_stream stream);
+
+/*
  * tra_plan_status -- read and clear the current device's error word.  Call
  * after synchronising the streams that ran this library's kernels.  Returns
  * TRA_OK, TRA_ERR_TIMEOUT or TRA_ERR_DEVICE_CHECK (or TRA_ERR_CUDA if the

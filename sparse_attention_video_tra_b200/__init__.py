@@ -20,7 +20,7 @@ from dataclasses import dataclass
 __all__ = [
     "TraError", "PlanInfo", "Plan", "library_path", "load_library",
     "tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
-    "tra_radius_and_mask", "tra_attention", "tra_plan_status", "tra_status_string",
+    "tra_radius_and_mask", "tra_attention", "tra_calibrate_topk", "tra_plan_status", "tra_status_string",
     "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "TRA_FLAG_DISK", "tra_flag_tile_w",
 ]
 
@@ -108,6 +108,8 @@ def load_library() -> ctypes.CDLL:
     L.tra_radius_and_mask.restype = st
     L.tra_attention.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     L.tra_attention.restype = st
+    L.tra_calibrate_topk.argtypes = [vp, vp, vp, ctypes.c_double, i, vp, vp, vp]
+    L.tra_calibrate_topk.restype = st
     L.tra_plan_status.argtypes = [vp]
     L.tra_plan_status.restype = st
     L.tra_status_string.argtypes = [st]
@@ -160,6 +162,12 @@ def tra_radius_and_mask(plan, H_ptr, mask_ptr, mask_bytes, stream=0) -> None:
 
 def tra_attention(plan, q_ptr, k_ptr, v_ptr, mask_ptr, out_ptr, stream=0) -> None:
     _check("tra_attention", load_library().tra_attention(plan, q_ptr, k_ptr, v_ptr, mask_ptr, out_ptr, stream))
+
+
+def tra_calibrate_topk(plan, q_ptr, k_ptr, mass, query_tile_stride, H_ptr, k_out_ptr, stream=0) -> None:
+    _check("tra_calibrate_topk", load_library().tra_calibrate_topk(plan, q_ptr, k_ptr, float(mass),
+                                                                   int(query_tile_stride), H_ptr, k_out_ptr,
+                                                                   stream))
 
 
 def tra_plan_status(plan) -> int:
@@ -291,6 +299,21 @@ class Plan:
         tra_attention(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), mask.data_ptr(), out.data_ptr(),
                       self._stream(stream))
         return out
+
+    def calibrate_topk(self, q, k, mass, query_tile_stride=1, stream=None):
+        """Calibration workload: (H [heads, n_sample, 128] fp32, k [heads,
+        n_sample, 128] int32) for the queries of every query_tile_stride-th
+        tile; k_i = fewest top keys holding `mass` of the query's attention."""
+        import torch
+        i = self.info
+        self._rows(q, self.io_rows, "q")
+        self._rows(k, self.io_rows, "k")
+        n_sample = -(-i.n_tiles // int(query_tile_stride))
+        H = torch.empty(i.heads, n_sample, 128, dtype=torch.float32, device=q.device)
+        K = torch.empty(i.heads, n_sample, 128, dtype=torch.int32, device=q.device)
+        tra_calibrate_topk(self.handle, q.data_ptr(), k.data_ptr(), mass, query_tile_stride, H.data_ptr(),
+                           K.data_ptr(), self._stream(stream))
+        return H, K
 
     def status(self) -> int:
         return tra_plan_status(self.handle)

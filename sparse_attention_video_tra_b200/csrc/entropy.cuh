@@ -46,6 +46,61 @@ struct EntCfg {
 // on the FMA pipe (degree-4 polynomial, packed pairs), the rest on the MUFU unit
 constexpr int ENT_POLY_MOD = 3;
 
+// One key tile's contribution to a query row's online entropy statistics in
+// the log2 domain: m = running maximum of s*c, Z = sum 2^(s*c - m), A = sum
+// 2^(s*c - m) * (s*c - m); the entropy is then ln Z - ln2 * A / Z.  v holds the
+// row's 128 raw scores s of the tile; pad keys of edge tiles are dropped.
+template <int TWL>
+__device__ __forceinline__ void ent_tile_update(uint32_t (&v)[4][32], bool edge, int khv, int kwv, float c,
+                                                float& m, float& Z, float& A)
+{
+    if (edge) {                     // pad keys of edge tiles take no probability
+        uint32_t keep[4];
+        row_keep_bits<TWL>(0, khv - 1, 0, kwv - 1, keep);
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+            if (!(keep[i >> 5] & (1u << (i & 31)))) v[i >> 5][i & 31] = __float_as_uint(-1e30f);
+    }
+    // four independent max chains, then combine
+    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+        m4[i & 3] = max3(m4[i & 3], __uint_as_float(v[i >> 4][(2 * i) & 31]), __uint_as_float(v[i >> 4][(2 * i + 1) & 31]));
+    const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
+    if (mt > m) {
+        const float alpha = ex2(m - mt);
+        A = alpha * fmaf(m - mt, Z, A);
+        Z *= alpha;
+        m = mt;
+    }
+    // u = s*c - m (<= 0), e = 2^u; Z += e, A += e*u, all in packed pairs;
+    // four independent accumulator chains
+    const f2_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
+    f2_t z2[4] = {0ull, 0ull, 0ull, 0ull}, a2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const f2_t u2 = f2_fma(f2_pack(__uint_as_float(v[i >> 4][(2 * i) & 31]),
+                                       __uint_as_float(v[i >> 4][(2 * i + 1) & 31])), c2, nm2);
+        f2_t e2;
+        if (i % ENT_POLY_MOD == ENT_POLY_MOD - 1) {
+            e2 = ex2_poly4_pair(u2);
+        } else {
+            float u0, u1;
+            f2_unpack(u2, u0, u1);
+            e2 = f2_pack(ex2(u0), ex2(u1));
+        }
+        z2[i & 3] = f2_add(z2[i & 3], e2);
+        a2[i & 3] = f2_fma(e2, u2, a2[i & 3]);
+    }
+    const f2_t zs = f2_add(f2_add(z2[0], z2[1]), f2_add(z2[2], z2[3]));
+    const f2_t as = f2_add(f2_add(a2[0], a2[1]), f2_add(a2[2], a2[3]));
+    float zl, zh, al, ah;
+    f2_unpack(zs, zl, zh);
+    f2_unpack(as, al, ah);
+    Z += zl + zh;
+    A += al + ah;
+}
+
 template <int D, int TWL>
 __global__ void __launch_bounds__(352, 1)
 entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -172,51 +227,7 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_empty[bs]);
-            if (edge) {                     // pad keys of edge tiles take no probability
-                uint32_t keep[4];
-                row_keep_bits<TWL>(0, khv - 1, 0, kwv - 1, keep);
-#pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    if (!(keep[i >> 5] & (1u << (i & 31)))) v[i >> 5][i & 31] = __float_as_uint(-1e30f);
-            }
-            // four independent max chains, then combine
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-                m4[i & 3] = max3(m4[i & 3], __uint_as_float(v[i >> 4][(2 * i) & 31]), __uint_as_float(v[i >> 4][(2 * i + 1) & 31]));
-            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
-            if (mt > m) {
-                const float alpha = ex2(m - mt);
-                A = alpha * fmaf(m - mt, Z, A);
-                Z *= alpha;
-                m = mt;
-            }
-            // u = s*c - m (<= 0), e = 2^u; Z += e, A += e*u, all in packed pairs;
-            // four independent accumulator chains
-            const f2_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
-            f2_t z2[4] = {0ull, 0ull, 0ull, 0ull}, a2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const f2_t u2 = f2_fma(f2_pack(__uint_as_float(v[i >> 4][(2 * i) & 31]),
-                                               __uint_as_float(v[i >> 4][(2 * i + 1) & 31])), c2, nm2);
-                f2_t e2;
-                if (i % ENT_POLY_MOD == ENT_POLY_MOD - 1) {
-                    e2 = ex2_poly4_pair(u2);
-                } else {
-                    float u0, u1;
-                    f2_unpack(u2, u0, u1);
-                    e2 = f2_pack(ex2(u0), ex2(u1));
-                }
-                z2[i & 3] = f2_add(z2[i & 3], e2);
-                a2[i & 3] = f2_fma(e2, u2, a2[i & 3]);
-            }
-            const f2_t zs = f2_add(f2_add(z2[0], z2[1]), f2_add(z2[2], z2[3]));
-            const f2_t as = f2_add(f2_add(a2[0], a2[1]), f2_add(a2[2], a2[3]));
-            float zl, zh, al, ah;
-            f2_unpack(zs, zl, zh);
-            f2_unpack(as, al, ah);
-            Z += zl + zh;
-            A += al + ah;
+            ent_tile_update<TWL>(v, edge, khv, kwv, c, m, Z, A);
         }
         if (ok) {
             const float H = logf(Z) - 0.69314718055994531f * (A / Z) + corr;

@@ -16,6 +16,7 @@
 #include "radius_mask.cuh"
 #include "entropy.cuh"
 #include "attention.cuh"
+#include "topk.cuh"
 
 namespace {
 
@@ -109,6 +110,17 @@ tra_status run_entropy(const tra::Geom& G, const CUtensorMap& q, const CUtensorM
     auto kern = tra::entropy_kernel<D, TWL>;
     if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
     kern<<<dim3((G.nQ + 1) / 2, G.G), C::THREADS, C::SMEM, st>>>(q, k, G, stride, corr, H);
+    return launch_status();
+}
+
+template <int D, int TWL>
+tra_status run_topk(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, int stride, int n_sample,
+                    float mass, float* H, int* K, cudaStream_t st)
+{
+    using C = tra::TopkCfg<D>;
+    auto kern = tra::topk_kernel<D, TWL>;
+    if (!set_smem(kern, C::SMEM)) return TRA_ERR_CUDA;
+    kern<<<dim3(n_sample, G.G), C::THREADS, C::SMEM, st>>>(q, k, G, stride, n_sample, mass, H, K);
     return launch_status();
 }
 
@@ -218,6 +230,31 @@ extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k,
     const bool ob = (plan->flags & TRA_FLAG_OUT_BF16) != 0;
     const bool disk = G.disk != 0;
     return dispatch_attention(G, ob, disk, mq, mk, mv, m, out, st);
+}
+
+extern "C" tra_status tra_calibrate_topk(tra_plan plan, const void* q, const void* k, double mass,
+                                         int query_tile_stride, float* H_out, int* k_out, tra_stream stream)
+{
+    if (!plan || !q || !k || !H_out || !k_out) return TRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(H_out, 4) || !aligned(k_out, 4)) return TRA_ERR_INVALID_ARG;
+    if (!(mass > 0.0 && mass < 1.0) || query_tile_stride < 1) return TRA_ERR_INVALID_ARG;
+    const tra::Geom& G = plan->geom;
+    const int n_sample = (G.nQ + query_tile_stride - 1) / query_tile_stride;
+    CUtensorMap mq, mk;
+    if (!make_input_map(&mq, q, G) || !make_input_map(&mk, k, G)) return TRA_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    const float m = (float)mass;
+    switch (G.D * 100 + G.tw_log2) {
+        case 6402: return run_topk<64, 2>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 6403: return run_topk<64, 3>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 6404: return run_topk<64, 4>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 6405: return run_topk<64, 5>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 12802: return run_topk<128, 2>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 12803: return run_topk<128, 3>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 12804: return run_topk<128, 4>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+        case 12805: return run_topk<128, 5>(G, mq, mk, query_tile_stride, n_sample, m, H_out, k_out, st);
+    }
+    return TRA_ERR_UNSUPPORTED;
 }
 
 extern "C" tra_status tra_plan_status(tra_plan plan)
