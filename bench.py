@@ -282,6 +282,9 @@ def run_tra(args, rank, world):
     if args.heads:
         import dataclasses
         wl = dataclasses.replace(wl, heads=args.heads, name=wl.name.replace(f"{wl.heads} heads", f"{args.heads} heads"))
+    if args.retained:
+        import dataclasses
+        wl = dataclasses.replace(wl, target_retained=float(args.retained), b=None)
     calls = args.calls if args.calls else (10 if args.workload == "wan720" else 1)
     total_heads, workload_name = wl.heads, wl.name
     if args.shard == "heads":
@@ -499,6 +502,8 @@ def main(argv=None):
     ap.add_argument("--shard", default="replica", choices=["replica", "heads"],
                     help="replica: every rank runs the whole workload (weak scaling); "
                          "heads: the workload's heads are split over the ranks (strong scaling)")
+    ap.add_argument("--retained", type=float, default=0.0,
+                    help="target retained fraction for calibrating b (0 = the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
