@@ -209,6 +209,61 @@ def oracle_sample(wl, b, budget_s: float, rng_seed: int, heads=(0,), device="cud
                     "retained_pairs": pairs}
 
 
+def oracle_parity(run, wl, n_queries: int = 256, seed: int = 77):
+    """Part of the CPU-baseline leg: the fp64 oracle on a random sample of head
+    0's queries against this run's GPU results at full size -- entropy
+    (relative error), radii from the GPU's entropies (mismatches; bit-exact
+    expected) and attention rows of call 0 with those radii (max/mean abs)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    T, H, W, d, N = wl.T, wl.H, wl.W, wl.d, wl.N
+    i = run.info
+    run.run_attention(0)
+    torch.cuda.synchronize()
+    # tile-major row -> natural token for head 0
+    p = np.arange(i.N_pad)
+    tile, inn = p // 128, p % 128
+    tpf = i.n_tiles_h * i.n_tiles_w
+    t, rem = tile // tpf, tile % tpf
+    hh = (rem // i.n_tiles_w) * i.tile_h + inn // i.tile_w
+    ww = (rem % i.n_tiles_w) * i.tile_w + inn % i.tile_w
+    valid = (hh < H) & (ww < W)
+    nat = np.where(valid, (t * H + hh) * W + ww, -1)
+    rows = np.sort(np.random.default_rng(seed).choice(np.nonzero(valid)[0], n_queries, replace=False))
+    queries = nat[rows]
+    order = np.argsort(queries)
+    rows, queries = rows[order], queries[order]
+
+    # natural-order head-0 inputs (bf16 bit patterns)
+    from sparse_attention_video_tra_b200 import Plan
+    p1 = Plan(T, H, W, 1, d, wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, run.plan.flags)
+    nq = torch.empty((1, N, d), dtype=torch.bfloat16, device="cuda")
+    bits = []
+    for x in (run.q, run.k, run.v[0]):
+        p1.permute(x[:1].contiguous(), nq, False)
+        bits.append(nq.cpu().view(torch.int16).numpy().view(np.uint16).copy())
+    p1.close()
+    qb, kb, vb = bits
+    Hg = run.H[0].cpu().numpy()[rows]
+    if wl.key_stride == 1:
+        Hr = oracle.entropy(qb, kb, 1, (T, H, W), d, queries=queries)
+    else:
+        Hr = _oracle_entropy_tiled(oracle, qb, kb, 1, wl, queries)
+    rad = run.plan.mask_views(run.mask)[0][0].cpu().numpy()
+    r_ref, _, _ = oracle.radius(Hg, 1, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, queries=queries)
+    r_all = np.zeros(N, np.int32)
+    r_all[nat[valid]] = rad[valid]
+    O = oracle.attention(qb, kb, vb, r_all, 1, (T, H, W), d, wl.gamma, wl.Rt, queries=queries)
+    Og = run.out[0].float().cpu().numpy()[rows]
+    err = np.abs(Og - O)
+    return {"queries": int(n_queries), "head": 0,
+            "entropy_max_rel": float(np.max(np.abs(Hg - Hr) / np.maximum(np.abs(Hr), 1.0))),
+            "radius_mismatches": int(np.sum(rad[rows] != r_ref)),
+            "attention_max_abs": float(err.max()), "attention_mean_abs": float(err.mean()),
+            "tolerances": {"entropy_rel": 1e-3, "radius": "bit-exact", "attention_max_abs": 1e-2,
+                           "attention_mean_abs": 1e-3}}
+
+
 def _oracle_entropy_tiled(oracle, qb, kb, G, wl, idx):
     # key subsampling is defined on the library's key tiles: pass the plan's tile shape
     from sparse_attention_video_tra_b200 import Plan
@@ -371,7 +426,8 @@ def run_tra(args, rank, world):
         v, desc = oracle_sample(wl, run.b, args.cpu_budget, 4321)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": desc["threads"], "kind": "oracle",
                "sample": f"{desc['queries']} random queries of head 0: entropy+radius+attention in fp64, "
-                         f"{desc['seconds']} s"}
+                         f"{desc['seconds']} s",
+               "parity": oracle_parity(run, wl)}
 
     e2e = None if args.no_e2e else run_e2e(run, wl, calls, args, world)
     b_used, retained = run.b, run.retained_fraction_now()

@@ -208,7 +208,10 @@ TRA_API tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void* m
  * rounded to bf16 and O is normalised by the sum of those rounded values.
  *   q, k, v    device bf16 [heads][N_pad][d] tile-major, 16-byte aligned,
  *              finite pad rows
- *   mask       the buffer written by tra_radius_and_mask for this plan
+ *   mask       the buffer written by tra_radius_and_mask for this plan; a
+ *              tile count outside [0, list_cap] or a listed tile no query of
+ *              the tile can reach is recorded as TRA_ERR_DEVICE_CHECK (read by
+ *              tra_plan_status) and never dereferenced
  *   out        device [heads][N_pad][d] tile-major, fp32 (bf16 when the plan
  *              has TRA_FLAG_OUT_BF16); pad rows unspecified
  * With TRA_FLAG_NATURAL q, k, v and out are [heads][N][d] in natural token

@@ -128,7 +128,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const bool hasB = qb < G.nQ;
     const int32_t* counts = reinterpret_cast<const int32_t*>(mask + G.off_count) + (size_t)g * G.nQ;
     const uint16_t* lists = reinterpret_cast<const uint16_t*>(mask + G.off_list) + (size_t)g * G.nQ * G.list_cap;
-    const int nA = counts[qa], nB = hasB ? counts[qb] : 0;
+    int nA = counts[qa], nB = hasB ? counts[qb] : 0;
+    // the mask buffer is caller memory: a count outside [0, list_cap] is an
+    // error (recorded; this CTA then does nothing)
+    if (nA < 0 || nA > G.list_cap || nB < 0 || nB > G.list_cap) {
+        if (threadIdx.x == 0) atomicOr(&g_tra_error, TRA_ERRBIT_CHECK);
+        nA = 0;
+        nB = 0;
+    }
     const int ta = qa / G.tiles_per_frame;
     const int base = max(0, ta - G.rte) * G.tiles_per_frame;   // first key tile either list can hold
 
@@ -139,6 +146,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool isB = i >= nA;
         const int e = isB ? lists[(size_t)qb * G.list_cap + (i - nA)] : lists[(size_t)qa * G.list_cap + i];
         const int bit = (e & 0x7fff) - base;
+        // a key tile no query of the pair can reach is an error: recorded, skipped
+        if (bit < 0 || bit >= 32 * L.bw || (e & 0x7fff) >= G.nQ) {
+            atomicOr(&g_tra_error, TRA_ERRBIT_CHECK);
+            continue;
+        }
         atomicOr(&bits[(isB ? 1 : 0) * L.bw + (bit >> 5)], 1u << (bit & 31));
         if (e & 0x8000) atomicOr(&bits[(isB ? 3 : 2) * L.bw + (bit >> 5)], 1u << (bit & 31));
     }

@@ -28,6 +28,7 @@ namespace tra {
 // clipped neighbourhood count c(r) of the query at (t, h, w): per frame the
 // Chebyshev square is a clipped rectangle; the disk sums, key row by key row,
 // the clipped width 2*isqrt(s^2 - dh^2) + 1
+template <bool DISK>
 __device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int w, int r)
 {
     long long c = 0;
@@ -35,7 +36,7 @@ __device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int 
         const int m = (t + dl < G.T ? 1 : 0) + (dl > 0 && t - dl >= 0 ? 1 : 0);
         if (m == 0) break;                         // farther frames are out of the grid too
         const int s = halfwidth(r, G.g[dl]);
-        if (G.disk) {
+        if constexpr (DISK) {
             const int sc = min(s, TRA_DISK_S_CLAMP);
             const int hl = max(0, h - sc), hh = min(G.H - 1, h + sc);
             long long X = 0;
@@ -62,6 +63,7 @@ __device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
     return (long long)ceil(B);
 }
 
+template <bool DISK>
 __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
                                                           uint8_t* __restrict__ mask)
 {
@@ -100,10 +102,10 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         int lo = 0, hi = G.r_cap;
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (nbr_count(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+            if (nbr_count<DISK>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
         }
         r = lo;
-        c = nbr_count(G, t, h, w, r);
+        c = nbr_count<DISK>(G, t, h, w, r);
     }
     reinterpret_cast<int32_t*>(mask + G.off_radius)[row] = r;
 
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         for (int tr = r_lo; tr <= r_hi; ++tr) {
             const bool in = rl <= tr && tr <= rh;
             int c_lo = cl, c_hi = ch;
-            if (G.disk && in) {
+            if (DISK && in) {
                 // the disk is widest on the tile row's key row nearest to h
                 const int s = min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP);
                 const int k0 = tr * G.th, k1 = min(G.H - 1, k0 + G.th - 1);
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
 
     // ---- disk: a listed tile is full iff, for every valid query, its valid
     // key rectangle's farthest corner lies in the disk (the disk is convex)
-    if (G.disk) {
+    if constexpr (DISK) {
         for (int dl = 0; dl <= G.rte; ++dl) {
             if (!(t + dl < G.T || t - dl >= 0)) break;
             const int s = valid ? min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP) : 0;
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         const uint32_t fbits = s_fullbits[dl][tr];
         const int base = ((t0 + f) * G.nTh + tr) * G.nTw;
         for (int tc = lo; tc <= hi; ++tc) {
-            const bool full = G.disk ? ((fbits >> tc) & 1u) != 0
+            const bool full = DISK ? ((fbits >> tc) & 1u) != 0
                                      : (row_full && s_full[dl][2] <= tc && tc <= s_full[dl][3]);
             list[off++] = (uint16_t)((base + tc) | (full ? 0x8000 : 0));
         }
