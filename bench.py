@@ -462,31 +462,40 @@ def mask_algorithmic_bytes(run) -> float:
 def run_e2e(run, wl, calls, args, world):
     """The same metric through the public API with host buffers.  Per step:
     pinned host -> device copies of Q, K (natural token order) and of each
-    call's V, the hot path on a natural-layout plan (TRA_FLAG_NATURAL: the
+    call's V, the hot path on natural-layout plans (TRA_FLAG_NATURAL: the
     kernels read frame-major tensors through 4-D TMA boxes, no permute pass),
-    and each call's output back to pinned host memory.  Copies run on their
-    own streams: V of call c+1 goes up while call c computes, and the output
-    of call c comes down while call c+1 computes (V and outputs are double
-    buffered)."""
+    and each call's output back to pinned host memory.
+
+    Heads are independent problems, so the heads are split into chunks, each
+    with its own plan and mask buffer: the first chunk's entropy starts once
+    its own Q and K are up, and only the last chunk's output of the last call
+    is copied after the compute ends.  Copies run on their own streams: V of
+    call c+1 goes up while call c computes, and each chunk's output comes down
+    while the next chunk computes (V and outputs are double buffered)."""
     from sparse_attention_video_tra_b200 import Plan, TRA_FLAG_NATURAL
+    from sparse_attention_video_tra_b200.runner import shard_heads
     i = run.info
-    plan = Plan(wl.T, wl.H, wl.W, wl.heads, wl.d, wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin,
-                run.plan.flags | TRA_FLAG_NATURAL)
+    n_chunks = max(1, min(args.e2e_chunks, wl.heads))
+    chunks = [shard_heads(wl.heads, n_chunks, c) for c in range(n_chunks)]
+    plans = [Plan(wl.T, wl.H, wl.W, cnt, wl.d, wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin,
+                  run.plan.flags | TRA_FLAG_NATURAL) for _, cnt in chunks]
     shape = (i.heads, i.N, i.d)
     hq = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     hk = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     hv = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
-    ho = torch.empty(shape, dtype=plan.out_dtype, pin_memory=True)
+    ho = torch.empty(shape, dtype=plans[0].out_dtype, pin_memory=True)
     tmp = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
     run.plan.permute(run.q, tmp, False); hq.copy_(tmp)
     run.plan.permute(run.k, tmp, False); hk.copy_(tmp)
     run.plan.permute(run.v[0], tmp, False); hv.copy_(tmp)
     del tmp
-    dq, dk = plan.new_input(), plan.new_input()
-    dv = [plan.new_input(), plan.new_input()]
-    do = [plan.new_out(), plan.new_out()]
-    dH = plan.new_entropy()
-    dmask = plan.new_mask()
+    dq = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    dk = torch.empty_like(dq)
+    dv = [torch.empty_like(dq), torch.empty_like(dq)]
+    do = [torch.empty(shape, dtype=plans[0].out_dtype, device="cuda") for _ in range(2)]
+    dH = torch.empty((i.heads, i.N), dtype=torch.float32, device="cuda")
+    dmask = [p.new_mask() for p in plans]
+    sl = [slice(g0, g0 + cnt) for g0, cnt in chunks]
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()                       # noqa: E731
@@ -494,15 +503,18 @@ def run_e2e(run, wl, calls, args, world):
     def step():
         start = ev(); start.record(comp)
         s_in.wait_event(start)
+        qk_in = []
         with torch.cuda.stream(s_in):
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            qk_in = ev(); qk_in.record(s_in)
-        comp.wait_event(qk_in)
-        plan.entropy(dq, dk, dH, wl.key_stride, stream=comp)
-        plan.radius_and_mask(dH, dmask, stream=comp)
+            for h in sl:
+                dq[h].copy_(hq[h], non_blocking=True)
+                dk[h].copy_(hk[h], non_blocking=True)
+                qk_in.append(ev()); qk_in[-1].record(s_in)
+        for p, h, m, e in zip(plans, sl, dmask, qk_in):
+            comp.wait_event(e)
+            p.entropy(dq[h], dk[h], dH[h], wl.key_stride, stream=comp)
+            p.radius_and_mask(dH[h], m, stream=comp)
         v_free = [start, start]                            # buffer b may be refilled
-        o_free = [start, start]                            # buffer b may be rewritten
+        o_free = [[start] * n_chunks for _ in range(2)]    # chunk of buffer b may be rewritten
         last = start
         for c in range(calls):
             b = c & 1
@@ -511,16 +523,17 @@ def run_e2e(run, wl, calls, args, world):
                 dv[b].copy_(hv, non_blocking=True)
                 v_in = ev(); v_in.record(s_in)
             comp.wait_event(v_in)
-            comp.wait_event(o_free[b])
-            plan.attention(dq, dk, dv[b], dmask, do[b], stream=comp)
-            done = ev(); done.record(comp)
+            for q, (p, h, m) in enumerate(zip(plans, sl, dmask)):
+                comp.wait_event(o_free[b][q])
+                p.attention(dq[h], dk[h], dv[b][h], m, do[b][h], stream=comp)
+                done = ev(); done.record(comp)
+                s_out.wait_event(done)
+                with torch.cuda.stream(s_out):
+                    ho[h].copy_(do[b][h], non_blocking=True)
+                    out_done = ev(); out_done.record(s_out)
+                o_free[b][q] = out_done
+                last = out_done
             v_free[b] = done
-            s_out.wait_event(done)
-            with torch.cuda.stream(s_out):
-                ho.copy_(do[b], non_blocking=True)
-                out_done = ev(); out_done.record(s_out)
-            o_free[b] = out_done
-            last = out_done
         comp.wait_event(last)
 
     for _ in range(args.warmup):
@@ -534,16 +547,18 @@ def run_e2e(run, wl, calls, args, world):
     e1.record(comp)
     torch.cuda.synchronize()
     barrier(world)
-    if plan.status() != 0:
+    if any(p.status() != 0 for p in plans):
         raise RuntimeError("device error word set during the end-to-end run")
     secs = e0.elapsed_time(e1) / 1000.0
     val = aggregate(run.attention_flops() * calls * args.steps, secs, world) / 1e12
     nbytes = i.heads * i.N * i.d * 2
     obytes = i.heads * i.N * i.d * ho.element_size()
-    plan.close()
+    for p in plans:
+        p.close()
     return {"value": round(val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": nbytes * (2 + calls),
             "d2h_bytes_per_step": obytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3),
-            "layout": "natural [heads][T][H][W][d]; copies overlapped with compute on two copy streams"}
+            "head_chunks": n_chunks,
+            "layout": "natural [heads][T][H][W][d]; heads in chunks, copies overlapped with compute on two copy streams"}
 
 
 def main(argv=None):
@@ -561,6 +576,8 @@ def main(argv=None):
     ap.add_argument("--retained", type=float, default=0.0,
                     help="target retained fraction for calibrating b (0 = the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="head chunks of the end-to-end leg (each its own plan; copies overlap the other chunks)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args(argv)
