@@ -140,6 +140,19 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- profiles
+ROOFLINE_KERNEL = "attention_kernel"     # the dominant kernel; its ncu summary is profiles/<kernel>_<workload>_*
+
+
+def source_sha256() -> str:
+    """sha256 over every file of the kernel source directory, in name order."""
+    from sparse_attention_video_tra_b200.build import CSRC
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        h.update(open(os.path.join(CSRC, f), "rb").read())
+    return h.hexdigest()
+
+
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source (else None)."""
@@ -151,12 +164,7 @@ def recorded_traffic(kernel: str, workload: str):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    from sparse_attention_video_tra_b200.build import CSRC
-    import hashlib
-    h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
-        h.update(open(os.path.join(CSRC, f), "rb").read())
-    if kv.get("source_sha256") != h.hexdigest():
+    if kv.get("source_sha256") != source_sha256():
         return None
     try:
         return float(kv["dram_bytes_per_launch"])
@@ -406,8 +414,8 @@ def run_tra(args, rank, world):
     achieved = flops / avg_call_s / 1e12
     peak = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     computed = run.computed_pairs()
-    traffic = recorded_traffic("attention", args.workload)
-    roofline = {"bound": "tensor", "kernel": "tra::attention_kernel", "achieved": round(achieved, 2),
+    traffic = recorded_traffic(ROOFLINE_KERNEL, args.workload)
+    roofline = {"bound": "tensor", "kernel": "tra::" + ROOFLINE_KERNEL, "achieved": round(achieved, 2),
                 "peak": peak, "peak_kind": f"{pk_kind} bf16 sustained", "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "computed_tile_tflops": round(4.0 * wl.d * computed / avg_call_s / 1e12, 2),

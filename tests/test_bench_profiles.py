@@ -1,0 +1,44 @@
+"""Host checks of the bench's roofline bookkeeping: the committed ncu traffic
+summary of the dominant kernel is found under the name the bench looks up,
+and its DRAM bytes are reported only while the kernel source it was taken on
+is unchanged."""
+import os
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _fields(path):
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    return kv
+
+
+def test_traffic_summary_exists_under_the_bench_kernel_name():
+    path = os.path.join(ROOT, "profiles", f"{bench.ROOFLINE_KERNEL}_wan720_traffic.txt")
+    assert os.path.exists(path)
+    kv = _fields(path)
+    assert kv["kernel"] == bench.ROOFLINE_KERNEL and kv["workload"] == "wan720"
+    # the per-launch figure is the captured one scaled by the units (heads): 40 of the capture's
+    assert float(kv["dram_bytes_per_launch"]) == float(kv["captured_dram_bytes"]) * 40 / int(kv["captured_heads"])
+    got = bench.recorded_traffic(bench.ROOFLINE_KERNEL, "wan720")
+    if kv["source_sha256"] == bench.source_sha256():
+        assert got == float(kv["dram_bytes_per_launch"])
+    else:
+        assert got is None
+
+
+def test_stale_or_missing_summary_reports_no_traffic(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic(bench.ROOFLINE_KERNEL, "wan720") is None
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / f"{bench.ROOFLINE_KERNEL}_wan720_traffic.txt").write_text(
+        "source_sha256: 0000\ndram_bytes_per_launch: 123\n")
+    assert bench.recorded_traffic(bench.ROOFLINE_KERNEL, "wan720") is None
+    (tmp_path / "profiles" / f"{bench.ROOFLINE_KERNEL}_wan720_traffic.txt").write_text(
+        f"source_sha256: {bench.source_sha256()}\ndram_bytes_per_launch: 123\n")
+    assert bench.recorded_traffic(bench.ROOFLINE_KERNEL, "wan720") == 123.0
