@@ -107,7 +107,9 @@ def least_padding_tile(H, W):
         nTh, nTw = -(-H // th), -(-W // tw)
         if nTw > 32 or nTh > 64:
             continue
-        key = (nTh * nTw, -tw)
+        # least padding; a tie goes to the tile whose long side runs along
+        # the frame's short side (the taller tile when H <= W)
+        key = (nTh * nTw, tw if H <= W else -tw)
         if best is None or key < best[0]:
             best = (key, th, tw)
     return best[1], best[2]
@@ -145,10 +147,15 @@ def test_forced_tile_width():
 
 
 def test_workload_tiles_match_the_documented_choice():
-    # tiny: (1,8,16) padded x2; Wan-480p: (1,32,4) x1.067; 720p: (1,8,16) x1.067
-    assert tra.Plan(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8).info.tile_w == 16
+    # least padding first; on a tie the tile's long side runs along the
+    # frame's short side.  tiny: (1,16,8) padded x2 (ties with (1,8,16));
+    # Wan-480p: (1,32,4) x1.067; 720p: (1,16,8) x1.067 (ties with (1,8,16))
+    assert tra.Plan(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8).info.tile_w == 8
     wan480 = tra.Plan(21, 30, 52, 12, 128, 1.0, 0.0, 0.8, 6, 8).info
     assert (wan480.tile_h, wan480.tile_w) == (32, 4)
     assert math.isclose(wan480.N_pad / wan480.N, 1664 / 1560)
     wan720 = tra.Plan(21, 45, 80, 40, 128, 1.0, 0.0, 0.8, 6, 8).info
-    assert (wan720.tile_h, wan720.tile_w) == (8, 16) and wan720.N_pad == 21 * 3840
+    assert (wan720.tile_h, wan720.tile_w) == (16, 8) and wan720.N_pad == 21 * 3840
+    # a portrait frame with the same tie takes the wider tile
+    portrait = tra.Plan(2, 80, 45, 1, 128, 1.0, 0.0, 0.8, 1, 8).info
+    assert (portrait.tile_h, portrait.tile_w) == (8, 16) and portrait.N_pad == 2 * 3840

@@ -25,7 +25,8 @@ pytestmark = pytest.mark.gpu
 
 # (T, H, W, heads, d, gamma, Rt, Bmin, forced tile_w or 0)
 CASES = [
-    (4, 8, 8, 2, 64, 0.7, 2, 8, 0),        # (1,8,16) tiles, half padding in w
+    (4, 8, 8, 2, 64, 0.7, 2, 8, 0),        # (1,16,8) tiles, half padding in h
+    (4, 8, 8, 2, 64, 0.7, 2, 8, 16),       # (1,8,16) tiles, half padding in w
     (3, 7, 9, 2, 128, 0.8, 1, 4, 0),       # one ragged tile per frame
     (5, 17, 23, 2, 128, 0.8, 3, 8, 0),     # ragged both ways
     (3, 30, 52, 1, 128, 0.8, 2, 8, 4),     # (1,32,4) tiles

@@ -21,13 +21,15 @@ pytestmark = pytest.mark.gpu
 
 # (T, H, W, heads, d, gamma, Rt, Bmin, forced tile_w or 0)
 CASES = [
-    (4, 8, 8, 2, 64, 0.7, 2, 8, 0),        # tiny workload shape: (1,8,16) tiles, half padding
+    (4, 8, 8, 2, 64, 0.7, 2, 8, 0),        # tiny workload shape: (1,16,8) tiles, half padding in h
+    (4, 8, 8, 2, 64, 0.7, 2, 8, 16),       # the same in (1,8,16) tiles, half padding in w
     (3, 7, 9, 2, 128, 0.8, 1, 4, 0),       # one ragged tile per frame
     (5, 17, 23, 2, 128, 0.8, 3, 8, 0),     # several tiles, ragged both ways
     (3, 30, 52, 1, 128, 0.8, 2, 8, 4),     # Wan-480p frame, (1,32,4) tiles
     (4, 19, 21, 2, 64, 0.6, 3, 2, 8),      # (1,16,8) tiles
     (3, 9, 70, 1, 128, 0.9, 2, 3, 32),     # (1,4,32) tiles
-    (2, 45, 80, 1, 128, 0.8, 1, 8, 16),    # 720p frame
+    (2, 45, 80, 1, 128, 0.8, 1, 8, 0),     # 720p frame, (1,16,8) tiles
+    (2, 45, 80, 1, 128, 0.8, 1, 8, 16),    # 720p frame, (1,8,16) tiles
 ]
 
 
