@@ -136,7 +136,9 @@ typedef struct {
  *             phi(delta) = exp(-gamma' delta) with gamma = exp(-gamma'))
  *   Rt        temporal reach in frames, 0 <= min(Rt, T-1) <= 31
  *   Bmin      smallest budget, 1 <= Bmin <= N
- *   flags     TRA_FLAG_*; 0 = defaults (tile shape with the least padding)
+ *   flags     TRA_FLAG_*; 0 = defaults (tile shape with the least padding; on
+ *             a tie the tile's long side runs along the frame's short side,
+ *             the taller tile when H <= W)
  * Returns TRA_ERR_INVALID_ARG for impossible values, TRA_ERR_UNSUPPORTED for
  * shapes the kernels do not handle (d not 64/128, H or W above 256, > 32 tile
  * columns per frame, > 32767 tiles per head, > 2048 key tiles listed per
