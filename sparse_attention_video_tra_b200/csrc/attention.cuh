@@ -368,10 +368,21 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!qvalid) { a_lo = 1; a_hi = 0; }
             // column bias (0 kept, -inf masked) as pairs; the row bias is added per key row
             f2_t colb[CP];
+            // disk: squared column distance dw^2 per key column (INT_MAX past the
+            // grid edge); key row a keeps the columns with dw^2 <= s^2 - dh^2
+            int cdw2[DISK ? TW : 1];
+            if constexpr (DISK) {
 #pragma unroll
-            for (int bp = 0; bp < CP; ++bp)
-                colb[bp] = f2_pack((2 * bp >= b_lo && 2 * bp <= b_hi) ? 0.f : -INFINITY,
-                                   (2 * bp + 1 >= b_lo && 2 * bp + 1 <= b_hi) ? 0.f : -INFINITY);
+                for (int b = 0; b < TW; ++b) {
+                    const int dw = w0 + b - wq;
+                    cdw2[b] = b < kwv ? dw * dw : INT_MAX;
+                }
+            } else {
+#pragma unroll
+                for (int bp = 0; bp < CP; ++bp)
+                    colb[bp] = f2_pack((2 * bp >= b_lo && 2 * bp <= b_hi) ? 0.f : -INFINITY,
+                                       (2 * bp + 1 >= b_lo && 2 * bp + 1 <= b_hi) ? 0.f : -INFINITY);
+            }
 
             const bool got = role_wait(&s_full[w], k & 1, G.wait_ns, s_abort);
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
@@ -388,21 +399,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const float rb = (a >= a_lo && a <= a_hi) ? -m_run : -INFINITY;
                 const f2_t rb2 = f2_pack(rb, rb);
                 if constexpr (DISK) {
-                    // the disk keeps, on key row a, the columns within
-                    // isqrt(s^2 - dh^2) of the query column
-                    int blo = b_lo, bhi = b_hi;
-                    if (!full) {
-                        const int dh = h0 + a - hq;
-                        const int half = dh * dh <= s * s ? isqrt_floor(s * s - dh * dh) : -1;
-                        blo = max(0, wq - half - w0);
-                        bhi = min(kwv - 1, wq + half - w0);
-                    }
+                    // the disk keeps (a, b) iff dh^2 + dw^2 <= s^2 (a full tile
+                    // keeps every valid column); the row bias is the FMA's addend
+                    const int dh = h0 + a - hq;
+                    const int thr = full ? INT_MAX - 1 : s * s - dh * dh;
 #pragma unroll
                     for (int bp = 0; bp < CP; ++bp) {
                         const int i = a * CP + bp, c = (2 * i) >> 5, o = (2 * i) & 31;
-                        const f2_t cb = f2_pack((2 * bp >= blo && 2 * bp <= bhi) ? 0.f : -INFINITY,
-                                                (2 * bp + 1 >= blo && 2 * bp + 1 <= bhi) ? 0.f : -INFINITY);
-                        x[i] = f2_add(f2_fma(f2_pack(__uint_as_float(v[c][o]), __uint_as_float(v[c][o + 1])), sc2, cb), rb2);
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c][o]), __uint_as_float(v[c][o + 1])), sc2, rb2), x0, x1);
+                        x[i] = f2_pack(cdw2[2 * bp] <= thr ? x0 : -INFINITY, cdw2[2 * bp + 1] <= thr ? x1 : -INFINITY);
                     }
                 } else {
 #pragma unroll

@@ -37,13 +37,16 @@ __device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int 
         if (m == 0) break;                         // farther frames are out of the grid too
         const int s = halfwidth(r, G.g[dl]);
         if constexpr (DISK) {
+            // key rows h - k (k <= up) and h + k (k <= dn) share the half-width
+            // isqrt(s^2 - k^2)
             const int sc = min(s, TRA_DISK_S_CLAMP);
-            const int hl = max(0, h - sc), hh = min(G.H - 1, h + sc);
+            const int up = min(sc, h), dn = min(sc, G.H - 1 - h);
+            const int kmax = max(up, dn), s2 = sc * sc;
             long long X = 0;
-            for (int hk = hl; hk <= hh; ++hk) {
-                const int dh = hk - h;
-                const int half = isqrt_floor(sc * sc - dh * dh);
-                X += min(G.W - 1, w + half) - max(0, w - half) + 1;
+            for (int k = 0; k <= kmax; ++k) {
+                const int half = isqrt_floor(s2 - k * k);
+                const int wid = min(G.W - 1, w + half) - max(0, w - half) + 1;
+                X += k == 0 ? wid : (k <= up ? wid : 0) + (k <= dn ? wid : 0);
             }
             c += m * X;
         } else {
@@ -63,15 +66,26 @@ __device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
     return (long long)ceil(B);
 }
 
+// Dynamic shared memory of the mask kernel, sized from the plan so that small
+// reaches keep many CTAs resident: per (frame distance, tile row) the active
+// column interval [lo, hi] and the disk's full-column bits, and per list row
+// (frame, tile row) its length.
+__host__ __device__ inline int mask_smem_bytes(int rte, int nTh)
+{
+    return (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
+}
+
 template <bool DISK>
 __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
                                                           uint8_t* __restrict__ mask)
 {
-    __shared__ int s_lo[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];
-    __shared__ int s_hi[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];
+    extern __shared__ int mask_smem[];
+    const int RS = G.nTh;                                         // stride of one frame distance
+    int* s_lo = mask_smem;                                        // [rte + 1][nTh]
+    int* s_hi = s_lo + (G.rte + 1) * RS;                          // [rte + 1][nTh]
+    uint32_t* s_fullbits = reinterpret_cast<uint32_t*>(s_hi + (G.rte + 1) * RS);   // disk: full tile columns
+    int* s_len = reinterpret_cast<int*>(s_fullbits + (G.rte + 1) * RS);            // [(2 rte + 1) nTh]
     __shared__ int s_full[TRA_MAX_RT_EFF + 1][4];
-    __shared__ uint32_t s_fullbits[TRA_MAX_RT_EFF + 1][TRA_MAX_TILES_H];   // disk: full tile columns per row
-    __shared__ int s_len[TRA_MAX_LIST_ROWS];
     __shared__ long long s_pairs[4];
     __shared__ int s_warp[4];
 
@@ -84,10 +98,10 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     const bool valid = h < G.H && w < G.W;
     const size_t row = (size_t)g * G.N_pad + (size_t)tile * 128 + tid;
 
-    for (int i = tid; i < (G.rte + 1) * TRA_MAX_TILES_H; i += 128) {
-        (&s_lo[0][0])[i] = 0x7fffffff;
-        (&s_hi[0][0])[i] = -1;
-        (&s_fullbits[0][0])[i] = 0xffffffffu;
+    for (int i = tid; i < (G.rte + 1) * RS; i += 128) {
+        s_lo[i] = 0x7fffffff;
+        s_hi[i] = -1;
+        s_fullbits[i] = 0xffffffffu;
     }
     if (tid < G.rte + 1) {
         s_full[tid][0] = -0x7fffffff; s_full[tid][1] = 0x7fffffff;
@@ -100,6 +114,18 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     if (valid) {
         const long long bh = budget_hat(G, Hent[io_row(G, g, t, h, w, tile * 128 + tid)]);
         int lo = 0, hi = G.r_cap;
+        if constexpr (DISK) {
+            // the disk lies inside the square of the same half-width, so its
+            // radius is at least the square's; search [r_sq, 2 r_sq + 2] when
+            // that bracket reaches the budget, else the rest up to r_cap
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (nbr_count<false>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+            }
+            const int r2 = min(G.r_cap, 2 * lo + 2);
+            if (nbr_count<true>(G, t, h, w, r2) >= bh) hi = r2;
+            else { lo = min(r2 + 1, G.r_cap); hi = G.r_cap; }
+        }
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
             if (nbr_count<DISK>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
@@ -159,8 +185,8 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
             const int lo = __reduce_min_sync(0xffffffffu, in ? c_lo : 0x7fffffff);
             const int hi = __reduce_max_sync(0xffffffffu, in ? c_hi : -1);
             if (lane == 0 && hi >= 0) {
-                atomicMin(&s_lo[dl][tr], lo);
-                atomicMax(&s_hi[dl][tr], hi);
+                atomicMin(&s_lo[dl * RS + tr], lo);
+                atomicMax(&s_hi[dl * RS + tr], hi);
             }
         }
     }
@@ -173,7 +199,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
             if (!(t + dl < G.T || t - dl >= 0)) break;
             const int s = valid ? min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP) : 0;
             for (int tr = 0; tr < G.nTh; ++tr) {
-                const int lo = s_lo[dl][tr], hi = s_hi[dl][tr];
+                const int lo = s_lo[dl * RS + tr], hi = s_hi[dl * RS + tr];
                 if (hi < 0) continue;
                 const int k0 = tr * G.th, k1 = min(G.H - 1, k0 + G.th - 1);
                 const int dh = max(abs(h - k0), abs(h - k1));
@@ -184,7 +210,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
                     const bool in = !valid || (long long)dh * dh + (long long)dw * dw <= (long long)s * s;
                     if (__all_sync(0xffffffffu, in)) bits |= 1u << tc;
                 }
-                if (lane == 0) atomicAnd(&s_fullbits[dl][tr], bits | ~(((2u << hi) - 1u) ^ ((1u << lo) - 1u)));
+                if (lane == 0) atomicAnd(&s_fullbits[dl * RS + tr], bits | ~(((2u << hi) - 1u) ^ ((1u << lo) - 1u)));
             }
         }
         __syncthreads();
@@ -196,7 +222,7 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     for (int i = tid; i < R; i += 128) {
         const int f = i / G.nTh, tr = i - f * G.nTh;
         const int dl = abs(t0 + f - t);
-        s_len[i] = s_hi[dl][tr] >= 0 ? s_hi[dl][tr] - s_lo[dl][tr] + 1 : 0;
+        s_len[i] = s_hi[dl * RS + tr] >= 0 ? s_hi[dl * RS + tr] - s_lo[dl * RS + tr] + 1 : 0;
     }
     __syncthreads();
     const int per = (R + 127) >> 7;
@@ -216,9 +242,9 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     for (int i = beg; i < end; ++i) {
         const int f = i / G.nTh, tr = i - f * G.nTh;
         const int dl = abs(t0 + f - t);
-        const int lo = s_lo[dl][tr], hi = s_hi[dl][tr];
+        const int lo = s_lo[dl * RS + tr], hi = s_hi[dl * RS + tr];
         const bool row_full = s_full[dl][0] <= tr && tr <= s_full[dl][1];
-        const uint32_t fbits = s_fullbits[dl][tr];
+        const uint32_t fbits = s_fullbits[dl * RS + tr];
         const int base = ((t0 + f) * G.nTh + tr) * G.nTw;
         for (int tc = lo; tc <= hi; ++tc) {
             const bool full = DISK ? ((fbits >> tc) & 1u) != 0

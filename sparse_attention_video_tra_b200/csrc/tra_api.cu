@@ -181,9 +181,9 @@ extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void
     if (mask_bytes < plan->mask_bytes) return TRA_ERR_WORKSPACE;
     const tra::Geom& G = plan->geom;
     if (G.disk)
-        tra::radius_mask_kernel<true><<<dim3(G.nQ, G.G), 128, 0, (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
+        tra::radius_mask_kernel<true><<<dim3(G.nQ, G.G), 128, tra::mask_smem_bytes(G.rte, G.nTh), (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
     else
-        tra::radius_mask_kernel<false><<<dim3(G.nQ, G.G), 128, 0, (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
+        tra::radius_mask_kernel<false><<<dim3(G.nQ, G.G), 128, tra::mask_smem_bytes(G.rte, G.nTh), (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
     return launch_status();
 }
 
