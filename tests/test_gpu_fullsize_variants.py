@@ -1,0 +1,107 @@
+"""Full-size parity of the plan variants at the Wan-720p bench shape
+(21x45x80, 40 heads, d=128, 15 % of pairs retained), through the same
+resident-input path the benchmark times:
+
+* the Euclidean disk (TRA_FLAG_DISK) against the oracle's metric 1 on
+  sampled queries and query tiles: radii and block-mask rows bit-exact,
+  attention within max-abs 1e-2 / mean-abs 1e-3;
+* the natural token order (TRA_FLAG_NATURAL) against the tile-major path:
+  entropies, mask buffer and outputs bit for bit.
+
+Definitions: "Token Radius Attention for Efficient Video Generation"
+(gist.science summary), section 2; the disk is Intuition II's circular
+neighbourhood."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_video_tra_b200 as tra
+from sparse_attention_video_tra_b200 import build as trabuild
+from sparse_attention_video_tra_b200 import synth
+from sparse_attention_video_tra_b200.runner import WorkloadRun
+import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def run():
+    trabuild.build()
+    r = WorkloadRun(synth.WORKLOADS["wan720"], calls=1)
+    r.run_entropy()
+    r.run_mask()
+    r.run_attention(0)
+    torch.cuda.synchronize()
+    assert r.plan.status() == 0
+    yield r
+
+
+def _plan(run, flags):
+    wl = run.wl
+    return tra.Plan(wl.T, wl.H, wl.W, wl.heads, wl.d, wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, flags)
+
+
+def test_wan720_full_size_disk(run):
+    wl, i = run.wl, run.info
+    T, H, W, d, N = wl.T, wl.H, wl.W, wl.d, wl.N
+    plan = _plan(run, tra.TRA_FLAG_DISK)
+    mask, out = plan.new_mask(), plan.new_out()
+    plan.radius_and_mask(run.H, mask)
+    plan.attention(run.q, run.k, run.v[0], mask, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    rng = np.random.default_rng(11)
+    sel = [0, wl.heads - 1]
+    G = len(sel)
+    nat = gh.tile_major_index(i)
+    bits = lambda x: gh.bf16_bits(gh.to_natural(x[sel], i))     # noqa: E731
+    qb, kb, vb = bits(run.q), bits(run.k), bits(run.v[0])
+    o = gh.to_natural(out[sel], i).float().cpu().numpy().reshape(G * N, d)
+    Hg = gh.to_natural(run.H[sel], i).cpu().numpy().reshape(G * N)
+    rad, cnt, pairs, lst = plan.mask_views(mask)
+    r_nat = np.zeros((G, N), np.int32)
+    r_nat[:, nat[nat >= 0]] = rad[sel].cpu().numpy()[:, nat >= 0]
+    r_nat = r_nat.reshape(-1)
+    queries = np.sort(rng.choice(G * N, size=24, replace=False))
+    r_ref, _, _ = oracle.radius(Hg[queries], G, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin,
+                                queries=queries, metric=oracle.DISK)
+    np.testing.assert_array_equal(r_nat[queries], r_ref)
+    Oref = oracle.attention(qb, kb, vb, r_nat, G, (T, H, W), d, wl.gamma, wl.Rt, queries=queries,
+                            metric=oracle.DISK)
+    gh.check_attention(o[queries], Oref)
+    for t in rng.choice(i.n_tiles, size=2, replace=False):
+        for gi, g in enumerate(sel):
+            row = oracle.block_mask(r_nat, G, (T, H, W), wl.gamma, wl.Rt, (i.tile_h, i.tile_w),
+                                    (i.tile_h, i.tile_w), qtiles=[gi * i.n_tiles + int(t)], metric=oracle.DISK)[0]
+            n = int(cnt[g, t])
+            e = lst[g, t, :n].cpu().numpy().view(np.uint16).astype(np.int64)
+            dense = np.zeros(i.n_tiles, np.uint8)
+            dense[e & 0x7FFF] = np.where(e & 0x8000, 3, 1)
+            np.testing.assert_array_equal(dense, row)
+            members = nat[t * 128:(t + 1) * 128]
+            members = members[members >= 0] + gi * N
+            _, c_mem, _ = oracle.radius(Hg[members], G, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin,
+                                        queries=members, metric=oracle.DISK)
+            assert int(pairs[g, t]) == int(c_mem.sum())
+    plan.close()
+
+
+def test_wan720_full_size_natural_layout_is_bit_identical(run):
+    wl, i = run.wl, run.info
+    plan = _plan(run, tra.TRA_FLAG_NATURAL)
+    q, k, v = (gh.to_natural(x, i).contiguous() for x in (run.q, run.k, run.v[0]))
+    Hn, mask, out = plan.new_entropy(), plan.new_mask(), plan.new_out()
+    plan.entropy(q, k, Hn, wl.key_stride)
+    plan.radius_and_mask(Hn, mask)
+    plan.attention(q, k, v, mask, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    assert torch.equal(gh.to_natural(run.H, i), Hn)
+    a, b = run.plan.mask_views(run.mask), plan.mask_views(mask)
+    for x, y in zip(a[:3], b[:3]):                    # radii, tile counts, pair sums
+        assert torch.equal(x, y)
+    listed = torch.arange(i.list_cap, device=a[1].device).view(1, 1, -1) < a[1].unsqueeze(-1)
+    assert torch.equal(a[3][listed], b[3][listed])    # every listed entry, full flags included
+    assert torch.equal(gh.to_natural(run.out, i), out)
+    plan.close()
