@@ -24,6 +24,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "tra_oracle.c")
 _OUT = os.path.join(_HERE, "_build", "libtra_oracle.so")
+# A prebuilt oracle library to load instead (the mutation tests point this at
+# copies of tra_oracle.c with a planted mistake).
+_OVERRIDE = os.environ.get("TRA_ORACLE_LIB")
 _lib = None
 
 _I64P = ctypes.POINTER(ctypes.c_int64)
@@ -33,17 +36,24 @@ _F64P = ctypes.POINTER(ctypes.c_double)
 _U8P = ctypes.POINTER(ctypes.c_uint8)
 
 
+def compile_source(src: str, out: str) -> str:
+    """gcc the oracle's C source `src` into the shared library `out`."""
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+           "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile tra_oracle.c into oracle/_build/libtra_oracle.so."""
+    if _OVERRIDE:
+        return _OVERRIDE
     if not force and os.path.exists(_OUT) and os.path.getmtime(_OUT) >= os.path.getmtime(_SRC):
         return _OUT
     os.makedirs(os.path.dirname(_OUT), exist_ok=True)
-    tmp = _OUT + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, _OUT)
-    return _OUT
+    return compile_source(_SRC, _OUT)
 
 
 def lib() -> ctypes.CDLL:
