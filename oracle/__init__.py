@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_token_mask.restype = ctypes.c_int
         L.oracle_block_mask.argtypes = [_I32P] + [ctypes.c_int] * 4 + [ctypes.c_double, ctypes.c_int, ctypes.c_int] + \
             [ctypes.c_int] * 4 + [_I64P, ctypes.c_int64, _U8P]
+        L.oracle_block_mask_sets.argtypes = [_I32P] + [ctypes.c_int] * 4 + [ctypes.c_double, ctypes.c_int, ctypes.c_int] + \
+            [ctypes.c_int] * 2 + [_I64P, ctypes.c_int64, ctypes.c_int, _U8P]
         L.oracle_entropy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 5 + \
             [ctypes.c_int] * 3 + [_I64P, ctypes.c_int64, _F64P]
         L.oracle_attention.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, _I32P] + [ctypes.c_int] * 5 + \
@@ -181,6 +183,62 @@ def block_mask(r, G, grid, gamma, Rt, qtile, ktile, qtiles=None, metric: int = C
     out = np.zeros((rows, nK), np.uint8)
     lib().oracle_block_mask(_ptr(rr, _I32P), G, T, H, W, gamma, Rt, metric, qth, qtw, kth, ktw,
                             qp, nq, _ptr(out, _U8P))
+    return out
+
+
+def query_groups(r, G, grid, tile):
+    """The radius-sorted query groups of TRA_FLAG_QSORT plans (a design of this
+    library, not of the pages).  Query tiles are (1, th, tw) boxes in the
+    tile-major order; tiles 2p and 2p+1 of a head form a pair.  The pair's
+    256 tile-major rows are ordered by (radius, row) with pad rows (outside the
+    grid, radius -1) first; the first 128 are the group of tile 2p, the rest
+    that of tile 2p+1.
+
+    r: int32 radii [G*N] in natural order.  Returns
+      perm    uint8 [G, nQ, 128]: pair-local row (0..255) of each group slot;
+      members int64 [G*nQ, 128]: the slot's query as g*N + n, -1 on pad rows."""
+    T, H, W = grid
+    th, tw = tile
+    nTh, nTw = -(-H // th), -(-W // tw)
+    nQ = T * nTh * nTw
+    assert nQ % 2 == 0, "pairs need an even number of query tiles"
+    N = T * H * W
+    rr = np.asarray(r, dtype=np.int64).reshape(G, N)
+    p = np.arange(nQ * 128)
+    tile, inn = p // 128, p % 128
+    t, rem = tile // (nTh * nTw), tile % (nTh * nTw)
+    h = (rem // nTw) * th + inn // tw
+    w = (rem % nTw) * tw + inn % tw
+    valid = (h < H) & (w < W)
+    nat = np.where(valid, (t * H + h) * W + w, -1)
+    perm = np.zeros((G, nQ, 128), np.uint8)
+    members = np.full((G * nQ, 128), -1, np.int64)
+    for g in range(G):
+        rad = np.where(valid, rr[g][np.maximum(nat, 0)], -1)
+        for a in range(0, nQ, 2):
+            rows = np.arange(a * 128, a * 128 + 256)
+            order = np.argsort(rad[rows], kind="stable")        # (radius, row): stable on row
+            for k in range(2):
+                sl = order[128 * k:128 * (k + 1)]
+                perm[g, a + k] = sl
+                src = nat[rows[sl]]
+                members[g * nQ + a + k] = np.where(src >= 0, g * N + src, -1)
+    return perm, members
+
+
+def block_mask_sets(r, G, grid, gamma, Rt, ktile, members, metric: int = CHEBYSHEV) -> np.ndarray:
+    """Block-mask rows of explicit query sets: members int64 [n_sets, set_size]
+    (g*N + n, -1 = empty slot), one head per set.  Returns uint8 [n_sets, nK]
+    with 0 / 1 / 3 as block_mask."""
+    T, H, W = grid
+    rr = np.ascontiguousarray(np.asarray(r, dtype=np.int32).reshape(-1))
+    mem = np.ascontiguousarray(np.asarray(members, dtype=np.int64))
+    n_sets, set_size = mem.shape
+    kth, ktw = ktile
+    nK = T * (-(-H // kth)) * (-(-W // ktw))
+    out = np.zeros((n_sets, nK), np.uint8)
+    lib().oracle_block_mask_sets(_ptr(rr, _I32P), G, T, H, W, gamma, Rt, metric, kth, ktw,
+                                 _ptr(mem, _I64P), n_sets, set_size, _ptr(out, _U8P))
     return out
 
 

@@ -284,6 +284,50 @@ void oracle_block_mask(const int32_t* r, int G, int T, int H, int W,
     }
 }
 
+/* Block mask of explicit query sets (the radius-sorted query groups of the  */
+/* library's TRA_FLAG_QSORT plans): set s holds the queries                  */
+/* members[s*set_size .. s*set_size + set_size) as g*N + n (-1: no query).   */
+/* For every key tile of the query set's head: 0 inactive, 1 active (some    */
+/* member keeps some valid key of it), 3 active and full (every member keeps */
+/* every valid key of it).  A set without members is all 0.  All members of */
+/* a set belong to one head.                                                 */
+void oracle_block_mask_sets(const int32_t* r, int G, int T, int H, int W,
+                            double gamma, int Rt, int metric, int kth, int ktw,
+                            const int64_t* members, int64_t n_sets, int set_size,
+                            uint8_t* out)
+{
+    grid_t gr = {T, H, W};
+    int rte = oracle_rt_eff(T, Rt);
+    int64_t N = (int64_t)T * H * W;
+    int knTh = (H + kth - 1) / kth, knTw = (W + ktw - 1) / ktw;
+    int64_t nK = (int64_t)T * knTh * knTw;
+    (void)G;
+
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t set = 0; set < n_sets; ++set) {
+        const int64_t* mem = members + set * set_size;
+        for (int64_t kb = 0; kb < nK; ++kb) {
+            int bt = (int)(kb / ((int64_t)knTh * knTw));
+            int bh = (int)((kb / knTw) % knTh), bw = (int)(kb % knTw);
+            int any = 0, all = 1, some = 0;
+            for (int m = 0; m < set_size; ++m) {
+                int64_t gi = mem[m];
+                if (gi < 0) continue;
+                some = 1;
+                int64_t g = gi / N, i = gi % N;
+                for (int jh = 0; jh < kth; ++jh) for (int jw = 0; jw < ktw; ++jw) {
+                    int hj = bh * kth + jh, wj = bw * ktw + jw;
+                    if (hj >= H || wj >= W) continue;
+                    int64_t j = ((int64_t)bt * H + hj) * W + wj;
+                    if (token_mask(&gr, gamma, rte, metric, i, j, r[g * N + i])) any = 1;
+                    else all = 0;
+                }
+            }
+            out[set * nK + kb] = (uint8_t)(some && any ? (all ? 3 : 1) : 0);
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* E1 / E2: per-query softmax entropy ([TRA] Intuition I, "Entropie-vers-    */
 /* Budget"; [TLDR] fused entropy extraction).                                */

@@ -1,0 +1,107 @@
+"""Pins for the oracle's radius-sorted query groups (the library's
+TRA_FLAG_QSORT plans; a scheduling design of this library, not of the pages)
+and for the block mask of explicit query sets.
+
+* Block masks of sets equal the tile block mask when the sets are the tiles
+  (two independent oracle paths), and a dense numpy brute force for arbitrary
+  sets (bruteforce.token_mask).
+* The two groups of a pair partition its 256 rows, every radius of the first
+  group is at most every radius of the second, equal radii keep row order,
+  and pad rows come first.
+* Token voting is an OR, so the union of the two groups' active tiles equals
+  the union of the pair's two tiles' active tiles."""
+import numpy as np
+import pytest
+
+import oracle
+import bruteforce as bf
+
+
+def _tile_members(G, grid, tile):
+    T, H, W = grid
+    th, tw = tile
+    nTh, nTw = -(-H // th), -(-W // tw)
+    nQ = T * nTh * nTw
+    N = T * H * W
+    mem = np.full((G * nQ, 128), -1, np.int64)
+    for g in range(G):
+        for a in range(nQ):
+            t, rem = a // (nTh * nTw), a % (nTh * nTw)
+            for i in range(128):
+                h = (rem // nTw) * th + i // tw
+                w = (rem % nTw) * tw + i % tw
+                if h < H and w < W:
+                    mem[g * nQ + a, i] = g * N + (t * H + h) * W + w
+    return mem
+
+
+@pytest.mark.parametrize("grid,tile,metric", [((4, 8, 8), (16, 8), oracle.CHEBYSHEV), ((3, 7, 9), (8, 16), oracle.CHEBYSHEV),
+                                              ((2, 9, 13), (4, 32), oracle.DISK)])
+def test_sets_equal_tiles_when_sets_are_tiles(grid, tile, metric):
+    T, H, W = grid
+    G, N = 2, T * H * W
+    r = np.random.default_rng(1).integers(0, 7, G * N).astype(np.int32)
+    mem = _tile_members(G, grid, tile)
+    a = oracle.block_mask_sets(r, G, grid, 0.8, 2, tile, mem, metric=metric)
+    b = oracle.block_mask(r, G, grid, 0.8, 2, tile, tile, metric=metric)
+    np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("disk", [False, True])
+def test_sets_equal_bruteforce(disk):
+    T, H, W, gamma, Rt = 3, 7, 9, 0.8, 1
+    N = T * H * W
+    rng = np.random.default_rng(2)
+    r = rng.integers(0, 6, N).astype(np.int32)
+    M = bf.token_mask(T, H, W, gamma, Rt, r, disk=disk)        # [N, N] keep
+    kt = (2, 4)
+    kid, nK = bf.tile_ids(T, H, W, *kt)
+    sets = np.full((6, 10), -1, np.int64)
+    for s in range(6):
+        k = rng.integers(1, 11)
+        sets[s, :k] = rng.choice(N, size=k, replace=False)
+    got = oracle.block_mask_sets(r, 1, (T, H, W), gamma, Rt, kt, sets,
+                                 metric=oracle.DISK if disk else oracle.CHEBYSHEV)
+    for s in range(6):
+        q = sets[s][sets[s] >= 0]
+        for kb in range(nK):
+            keys = np.nonzero(kid == kb)[0]
+            blk = M[np.ix_(q, keys)]
+            want = (3 if blk.all() else 1) if blk.any() else 0
+            assert got[s, kb] == want
+
+
+def test_groups_partition_pairs_sorted_by_radius():
+    T, H, W, G = 3, 20, 16, 2
+    tile = (16, 8)
+    N = T * H * W
+    r = np.random.default_rng(3).integers(0, 9, G * N).astype(np.int32)
+    perm, mem = oracle.query_groups(r, G, (T, H, W), tile)
+    nQ = perm.shape[1]
+    tm = _tile_members(G, (T, H, W), tile)
+    for g in range(G):
+        for a in range(0, nQ, 2):
+            both = np.concatenate([perm[g, a], perm[g, a + 1]]).astype(np.int64)
+            assert sorted(both.tolist()) == list(range(256))
+            pair_rows = np.concatenate([tm[g * nQ + a], tm[g * nQ + a + 1]])
+            rad = np.where(pair_rows >= 0, r[np.maximum(pair_rows, 0)], -1)
+            ordered = rad[both]
+            assert np.all(np.diff(ordered) >= 0)                     # sorted by radius (pads, -1, first)
+            for v in np.unique(ordered):
+                rows = both[ordered == v]
+                assert np.all(np.diff(rows) > 0)                     # ties keep row order
+            for k in range(2):
+                np.testing.assert_array_equal(mem[g * nQ + a + k], pair_rows[perm[g, a + k].astype(np.int64)])
+
+
+def test_group_union_equals_tile_union():
+    T, H, W, G = 3, 20, 16, 2
+    tile = (16, 8)
+    N = T * H * W
+    r = np.random.default_rng(4).integers(0, 9, G * N).astype(np.int32)
+    _, mem = oracle.query_groups(r, G, (T, H, W), tile)
+    grp = oracle.block_mask_sets(r, G, (T, H, W), 0.8, 2, tile, mem) > 0
+    til = oracle.block_mask(r, G, (T, H, W), 0.8, 2, tile, tile) > 0
+    np.testing.assert_array_equal(grp[0::2] | grp[1::2], til[0::2] | til[1::2])
+    # and sorting never adds work: the groups list at most as many tiles as the tiles do
+    assert grp.sum() <= til.sum()
