@@ -337,6 +337,22 @@ def _oracle_calibrate_b(oracle, wl, dev):
     return 0.5 * (lo + hi)
 
 
+def query_group_flags(mode: str, wl) -> int:
+    """TRA_FLAG_QSORT when asked for, or (auto) when the workload's frame has
+    an even number of tile columns, so that a pair of query tiles is two
+    side-by-side tiles (the plan refuses the flag otherwise)."""
+    from sparse_attention_video_tra_b200 import Plan, TRA_FLAG_QSORT, TraError
+    if mode == "off":
+        return 0
+    try:
+        Plan(wl.T, wl.H, wl.W, 1, wl.d, wl.a, 0.0, wl.gamma, wl.Rt, wl.Bmin, TRA_FLAG_QSORT).close()
+    except TraError:
+        if mode == "on":
+            raise
+        return 0
+    return TRA_FLAG_QSORT
+
+
 def run_tra(args, rank, world):
     sys.path.insert(0, ROOT)
     from sparse_attention_video_tra_b200 import Plan, synth
@@ -358,7 +374,8 @@ def run_tra(args, rank, world):
         if count == 0:
             raise SystemExit(f"rank {rank}: no heads left to shard ({wl.heads} heads over {world} ranks)")
         wl = dataclasses.replace(wl, heads=count)
-    run = WorkloadRun(wl, calls=calls, seed_offset=rank)
+    flags = query_group_flags(args.qsort, wl)
+    run = WorkloadRun(wl, calls=calls, seed_offset=rank, flags=flags)
     dev_idx = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
@@ -439,6 +456,8 @@ def run_tra(args, rank, world):
 
     e2e = None if args.no_e2e else run_e2e(run, wl, calls, args, world)
     b_used, retained = run.b, run.retained_fraction_now()
+    tile_desc = f"1x{run.info.tile_h}x{run.info.tile_w}"
+    groups_desc = "radius-sorted pairs (TRA_FLAG_QSORT)" if run.plan.qsort else "spatial tiles"
     del run
     sharded = args.shard == "heads"
     line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -452,6 +471,7 @@ def run_tra(args, rank, world):
                                        else f"independent head-batch replicas x{world}"),
                        "attention_calls_per_step": calls,
                        "a": wl.a, "b": round(b_used, 6), "gamma": wl.gamma, "Rt": wl.Rt, "Bmin": wl.Bmin,
+                       "tile": tile_desc, "query_groups": groups_desc,
                        "inputs": "resident in HBM, 774 MB per tensor (> L2); L2 flushed before every step"},
             "retained_fraction": round(retained, 5), "phases": phases, "step_tflops": round(step_tflops, 3),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
@@ -464,7 +484,8 @@ def mask_algorithmic_bytes(run) -> float:
     per tile count (4 B) and pair sum (8 B), 2 B per listed key tile."""
     i = run.info
     listed = int(run.plan.mask_views(run.mask)[1].sum().item())
-    return i.heads * i.N_pad * 8.0 + i.heads * i.n_tiles * 12.0 + 2.0 * listed
+    groups = i.heads * i.N_pad * 1.0 if run.plan.qsort else 0.0      # 1 B per group slot
+    return i.heads * i.N_pad * 8.0 + i.heads * i.n_tiles * 12.0 + 2.0 * listed + groups
 
 
 def run_e2e(run, wl, calls, args, world):
@@ -583,6 +604,9 @@ def main(argv=None):
                          "heads: the workload's heads are split over the ranks (strong scaling)")
     ap.add_argument("--retained", type=float, default=0.0,
                     help="target retained fraction for calibrating b (0 = the workload's own)")
+    ap.add_argument("--qsort", default="auto", choices=["auto", "on", "off"],
+                    help="radius-sorted query groups (TRA_FLAG_QSORT): auto = when the frame has an even "
+                         "number of tile columns")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=4,
                     help="head chunks of the end-to-end leg (each its own plan; copies overlap the other chunks)")

@@ -21,7 +21,8 @@ __all__ = [
     "TraError", "PlanInfo", "Plan", "library_path", "load_library",
     "tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
     "tra_radius_and_mask", "tra_attention", "tra_calibrate_topk", "tra_plan_status", "tra_status_string",
-    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "TRA_FLAG_DISK", "tra_flag_tile_w",
+    "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "TRA_FLAG_DISK", "TRA_FLAG_QSORT",
+    "tra_flag_tile_w",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,6 +34,7 @@ TRA_FLAG_DEBUG_NO_WAIT = 1 << 16
 TRA_FLAG_OUT_BF16 = 1 << 17
 TRA_FLAG_NATURAL = 1 << 18
 TRA_FLAG_DISK = 1 << 19
+TRA_FLAG_QSORT = 1 << 20
 STATUS_NAMES = {0: "TRA_OK", 1: "TRA_ERR_INVALID_ARG", 2: "TRA_ERR_UNSUPPORTED", 3: "TRA_ERR_WORKSPACE",
                 4: "TRA_ERR_CUDA", 5: "TRA_ERR_TIMEOUT", 6: "TRA_ERR_DEVICE_CHECK"}
 
@@ -52,7 +54,7 @@ class _Info(ctypes.Structure):
                 ("T", "H", "W", "heads", "d", "N", "N_pad", "tile_h", "tile_w", "n_tiles_h", "n_tiles_w",
                  "n_tiles", "rt_eff", "r_cap", "list_cap")] + \
                [(n, ctypes.c_size_t) for n in
-                ("mask_bytes", "off_radius", "off_tile_count", "off_tile_pairs", "off_list")]
+                ("mask_bytes", "off_radius", "off_tile_count", "off_tile_pairs", "off_list", "off_group")]
 
 
 @dataclass(frozen=True)
@@ -77,6 +79,7 @@ class PlanInfo:
     off_tile_count: int
     off_tile_pairs: int
     off_list: int
+    off_group: int
 
 
 def library_path() -> str:
@@ -245,6 +248,21 @@ class Plan:
     def new_mask(self, device="cuda"):
         import torch
         return torch.empty(self.info.mask_bytes, dtype=torch.uint8, device=device)
+
+    @property
+    def qsort(self) -> bool:
+        """Radius-sorted query groups (TRA_FLAG_QSORT)."""
+        return bool(self.flags & TRA_FLAG_QSORT)
+
+    def group_view(self, mask):
+        """TRA_FLAG_QSORT: uint8 [heads, n_tiles, 128], the pair row (0..255)
+        of each slot of each tile's query group."""
+        import torch
+        i = self.info
+        if not self.qsort:
+            raise ValueError("the plan has no query groups (TRA_FLAG_QSORT)")
+        n = i.heads * i.n_tiles * 128
+        return mask[i.off_group:i.off_group + n].view(torch.uint8).view(i.heads, i.n_tiles, 128)
 
     def mask_views(self, mask):
         """(radius [heads,N_pad] i32, tile_count [heads,n_tiles] i32,

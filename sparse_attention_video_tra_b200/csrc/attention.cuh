@@ -31,6 +31,11 @@
 //              it); the two tiles progress independently.
 //   warp 11    idle (completes the third warpgroup for register rebalancing:
 //              the softmax warpgroups run with 216 registers, warps 8-11 with 72).
+// With radius-sorted query groups the CTA takes two mask slots instead (slot s
+// of frames 2f and 2f+1), stages the Q tiles of both pairs in the idle K/V
+// rings and copies each slot's 128 query rows into slot order before the
+// roles start; each softmax thread then speaks for its slot's query and
+// writes that query's output row.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 // (P_A, P_B as bf16 pairs in the first 64 columns of S_A, S_B).
 #pragma once
@@ -124,7 +129,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     const int pair = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qa = 2 * pair, qb = 2 * pair + 1;
+    // the CTA's two query tiles, or with radius-sorted groups two mask slots of
+    // like size and heavily overlapping lists: slot s of frames 2f and 2f + 1
+    // (both small-radius groups or both large-radius ones, one frame apart),
+    // so that the two per-slot chains stay about equally long and interleave
+    const int tpf = G.tiles_per_frame;
+    const int qa = G.qsort ? 2 * (pair / tpf) * tpf + pair % tpf : 2 * pair;
+    const int qb = G.qsort ? qa + tpf : qa + 1;
     const bool hasB = qb < G.nQ;
     const int32_t* counts = reinterpret_cast<const int32_t*>(mask + G.off_count) + (size_t)g * G.nQ;
     const uint16_t* lists = reinterpret_cast<const uint16_t*>(mask + G.off_list) + (size_t)g * G.nQ * G.list_cap;
@@ -205,6 +216,42 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t* sK = smem + C::OFF_K;
     uint8_t* sV = smem + C::OFF_V;
     const int kbase = g * G.N_pad;
+    // radius-sorted query groups: row r of slot s holds pair row grp_s[r] of
+    // the pair (tiles s & ~1 and (s & ~1) + 1)
+    const uint8_t* grp_a = mask + G.off_group + ((size_t)g * G.nQ + qa) * 128;
+    const uint8_t* grp_b = grp_a + (size_t)(qb - qa) * 128;
+    if (G.qsort && n > 0) {
+        // Q of both pairs lands in the idle K and V rings (four tiles, one
+        // pair without slot B), then each slot's rows are copied into
+        // slot order (128-byte swizzle on both sides)
+        static_assert(C::OFF_V == C::OFF_K + C::KST * C::TILE && C::KST + C::VST >= 4, "staging space");
+        const int np = hasB ? 2 : 1;
+        if (warp == C::WARP_LOAD && lane == 0) {
+            prefetch_tmap(&tm_q);
+            mbar_arrive_expect_tx(q_full, 2 * np * C::TILE);
+            for (int k = 0; k < 2 * np; ++k) {
+                int tq, trq, tcq;
+                tile_coords(G, ((k < 2 ? qa : qb) & ~1) + (k & 1), tq, trq, tcq);
+#pragma unroll
+                for (int p = 0; p < C::NP; ++p)
+                    load_tile_panel(sK + k * C::TILE + p * C::PANEL, &tm_q, G, p, g, tq, trq, tcq, q_full);
+            }
+        }
+        if (role_wait(q_full, 0, G.wait_ns, s_abort)) {
+            constexpr int CH = D / 8;                           // 16-byte chunks of a row
+            for (int i = tid; i < 128 * np * CH; i += C::THREADS) {
+                const int d = i / CH, ch = i - d * CH;
+                const int l = d < 128 ? grp_a[d] : grp_b[d - 128];
+                const int st = (d < 128 ? 0 : 2) + (l >> 7);     // staged tile
+                const int sr = l & 127, dr = d & 127, pn = ch >> 3, cc = ch & 7;
+                *reinterpret_cast<uint4*>(sQ + (d >> 7) * C::TILE + pn * C::PANEL + dr * 128 + ((cc ^ (dr & 7)) << 4)) =
+                    *reinterpret_cast<const uint4*>(sK + st * C::TILE + pn * C::PANEL + sr * 128 +
+                                                    ((cc ^ (sr & 7)) << 4));
+            }
+        }
+        fence_proxy_async_smem();                               // generic smem writes -> tensor-core reads
+        __syncthreads();
+    }
 
     if (warp >= C::WARP_LOAD) {
       regs_dec<C::REGS_OTHER>();
@@ -212,14 +259,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ------------------------------------------------ TMA producer: Q_A, Q_B, K and V rings
         if (lane == 0 && n > 0) {
             prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
-            int tqa, trqa, tcqa, tqb, trqb, tcqb;
-            tile_coords(G, qa, tqa, trqa, tcqa);
-            tile_coords(G, hasB ? qb : qa, tqb, trqb, tcqb);
+            if (!G.qsort) {                                         // else staged and gathered above
+                mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
+                int tqa, trqa, tcqa, tqb, trqb, tcqb;
+                tile_coords(G, qa, tqa, trqa, tcqa);
+                tile_coords(G, hasB ? qb : qa, tqb, trqb, tcqb);
 #pragma unroll
-            for (int p = 0; p < C::NP; ++p) {
-                load_tile_panel(sQ + p * C::PANEL, &tm_q, G, p, g, tqa, trqa, tcqa, q_full);
-                if (hasB) load_tile_panel(sQ + C::TILE + p * C::PANEL, &tm_q, G, p, g, tqb, trqb, tcqb, q_full);
+                for (int p = 0; p < C::NP; ++p) {
+                    load_tile_panel(sQ + p * C::PANEL, &tm_q, G, p, g, tqa, trqa, tcqa, q_full);
+                    if (hasB) load_tile_panel(sQ + C::TILE + p * C::PANEL, &tm_q, G, p, g, tqb, trqb, tcqb, q_full);
+                }
             }
             int kiss = 0, viss = 0;
             for (int j = 0; j < n; ++j) {
@@ -328,14 +377,21 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int row = tid & 127;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t colS = col_s(w), colO = col_o(w);
-        const int qt = w ? qb : qa;
         const bool active = w == 0 || hasB;
+        // this thread's query: row `row` of tile qa / qb, or the pair row of
+        // its group slot (radius-sorted groups)
+        int qt = w ? qb : qa, qrow = row;
+        if (G.qsort && active) {
+            const int l = (w ? grp_b : grp_a)[row];
+            qt = (qt & ~1) + (l >> 7);
+            qrow = l & 127;
+        }
         int tq, trq, tcq;
         tile_coords(G, active ? qt : qa, tq, trq, tcq);
-        const int hq = trq * G.th + (row >> TWL);
-        const int wq = tcq * TW + (row & (TW - 1));
+        const int hq = trq * G.th + (qrow >> TWL);
+        const int wq = tcq * TW + (qrow & (TW - 1));
         const bool qvalid = active && hq < G.H && wq < G.W;
-        const int rq = qvalid ? reinterpret_cast<const int32_t*>(mask + G.off_radius)[kbase + qt * 128 + row] : -1;
+        const int rq = qvalid ? reinterpret_cast<const int32_t*>(mask + G.off_radius)[kbase + qt * 128 + qrow] : -1;
         uint16_t* my_tab = s_tab + w * (G.rte + 1) * 128;
         for (int dl = 0; dl <= G.rte; ++dl)
             my_tab[dl * 128 + row] = (uint16_t)(qvalid ? min(halfwidth(rq, G.g[dl]), TRA_DISK_S_CLAMP) : 0);
@@ -485,7 +541,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 __syncwarp();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 const bool store = !G.natural || qvalid;          // natural layout has no pad rows
-                const size_t orow = io_row(G, g, tq, hq, wq, qt * 128 + row) * D;
+                const size_t orow = io_row(G, g, tq, hq, wq, qt * 128 + qrow) * D;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];

@@ -20,6 +20,12 @@
 //      pair retained) are the intersection of per-query rectangles.
 //   4. The active tiles of the frames within Rt' are written in ascending
 //      tile order after a block-wide prefix sum over (frame, tile row).
+// With radius-sorted query groups (a scheduling choice of this library) each
+// CTA first finds the radii of both tiles of its pair (2p, 2p+1: side by side
+// in one tile row), orders the pair's 256 rows by (radius, row), and then
+// speaks for the 128 queries of its own group instead of its own tile's rows;
+// step 3 still holds because every member's rectangle contains its own tile
+// column, one of two adjacent columns of the same tile row.
 #pragma once
 #include "tra_common.cuh"
 
@@ -66,22 +72,53 @@ __device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
     return (long long)ceil(B);
 }
 
+// r = the smallest r in [0, r_cap] whose neighbourhood count reaches bh (the
+// count is monotone in r; r_cap when none does); c = that count.
+template <bool DISK>
+__device__ __forceinline__ int find_radius(const Geom& G, int t, int h, int w, long long bh, long long& c)
+{
+    int lo = 0, hi = G.r_cap;
+    if constexpr (DISK) {
+        // the disk lies inside the square of the same half-width, so its
+        // radius is at least the square's; search [r_sq, 2 r_sq + 2] when
+        // that bracket reaches the budget, else the rest up to r_cap
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (nbr_count<false>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+        }
+        const int r2 = min(G.r_cap, 2 * lo + 2);
+        if (nbr_count<true>(G, t, h, w, r2) >= bh) hi = r2;
+        else { lo = min(r2 + 1, G.r_cap); hi = G.r_cap; }
+    }
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (nbr_count<DISK>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+    }
+    c = nbr_count<DISK>(G, t, h, w, lo);
+    return lo;
+}
+
 // Dynamic shared memory of the mask kernel, sized from the plan so that small
 // reaches keep many CTAs resident: per (frame distance, tile row) the active
 // column interval [lo, hi] and the disk's full-column bits, and per list row
 // (frame, tile row) its length.
-__host__ __device__ inline int mask_smem_bytes(int rte, int nTh)
+// With radius-sorted groups it also holds the pair's 256 counts, radii and
+// the group order.
+__host__ __device__ inline int mask_smem_bytes(int rte, int nTh, bool qsort)
 {
-    return (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
+    return (qsort ? 256 * (8 + 4 + 4) : 0) + (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
 }
 
-template <bool DISK>
+template <bool DISK, bool QS>
 __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
                                                           uint8_t* __restrict__ mask)
 {
-    extern __shared__ int mask_smem[];
+    extern __shared__ __align__(16) long long mask_smem[];
     const int RS = G.nTh;                                         // stride of one frame distance
-    int* s_lo = mask_smem;                                        // [rte + 1][nTh]
+    long long* s_qc = mask_smem;                                  // QS: [256] counts of the pair's rows
+    int* s_qr = reinterpret_cast<int*>(s_qc + (QS ? 256 : 0));    // QS: [256] radii of the pair's rows
+    int* s_qp = s_qr + (QS ? 256 : 0);                            // QS: [256] pair rows in group order
+    int* s_lo = s_qp + (QS ? 256 : 0);                            // [rte + 1][nTh]
     int* s_hi = s_lo + (G.rte + 1) * RS;                          // [rte + 1][nTh]
     uint32_t* s_fullbits = reinterpret_cast<uint32_t*>(s_hi + (G.rte + 1) * RS);   // disk: full tile columns
     int* s_len = reinterpret_cast<int*>(s_fullbits + (G.rte + 1) * RS);            // [(2 rte + 1) nTh]
@@ -93,10 +130,6 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int t, trq, tcq;
     tile_coords(G, tile, t, trq, tcq);
-    const int h = trq * G.th + (tid >> G.tw_log2);
-    const int w = tcq * G.tw + (tid & (G.tw - 1));
-    const bool valid = h < G.H && w < G.W;
-    const size_t row = (size_t)g * G.N_pad + (size_t)tile * 128 + tid;
 
     for (int i = tid; i < (G.rte + 1) * RS; i += 128) {
         s_lo[i] = 0x7fffffff;
@@ -108,32 +141,52 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         s_full[tid][2] = -0x7fffffff; s_full[tid][3] = 0x7fffffff;
     }
 
-    // ---- budget and radius
-    int r = -1;
+    // ---- budget and radius of the query this thread speaks for: its own row
+    // of the tile, or (QS) a slot of the tile's radius-sorted group
+    int h, w, r = -1;
+    bool valid;
     long long c = 0;
-    if (valid) {
-        const long long bh = budget_hat(G, Hent[io_row(G, g, t, h, w, tile * 128 + tid)]);
-        int lo = 0, hi = G.r_cap;
-        if constexpr (DISK) {
-            // the disk lies inside the square of the same half-width, so its
-            // radius is at least the square's; search [r_sq, 2 r_sq + 2] when
-            // that bracket reaches the budget, else the rest up to r_cap
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (nbr_count<false>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+    if constexpr (!QS) {
+        h = trq * G.th + (tid >> G.tw_log2);
+        w = tcq * G.tw + (tid & (G.tw - 1));
+        valid = h < G.H && w < G.W;
+        if (valid) r = find_radius<DISK>(G, t, h, w, budget_hat(G, Hent[io_row(G, g, t, h, w, tile * 128 + tid)]), c);
+        reinterpret_cast<int32_t*>(mask + G.off_radius)[(size_t)g * G.N_pad + (size_t)tile * 128 + tid] = r;
+    } else {
+        // both tiles of the pair (tiles 2p, 2p+1 side by side in one tile row)
+        const int pb = tile & ~1;
+        for (int k = 0; k < 2; ++k) {
+            const int hk = trq * G.th + (tid >> G.tw_log2);
+            const int wk = (tcq - (tile & 1) + k) * G.tw + (tid & (G.tw - 1));
+            int rk = -1;
+            long long ck = 0;
+            if (hk < G.H && wk < G.W)
+                rk = find_radius<DISK>(G, t, hk, wk, budget_hat(G, Hent[io_row(G, g, t, hk, wk, (pb + k) * 128 + tid)]), ck);
+            s_qr[k * 128 + tid] = rk;
+            s_qc[k * 128 + tid] = ck;
+            if (pb + k == tile)
+                reinterpret_cast<int32_t*>(mask + G.off_radius)[(size_t)g * G.N_pad + (size_t)tile * 128 + tid] = rk;
+        }
+        __syncthreads();
+        // order the pair's rows by (radius, row); pad rows (radius -1) first
+        for (int k = 0; k < 2; ++k) {
+            const int l = k * 128 + tid, rl = s_qr[l];
+            int rank = 0;
+            for (int j = 0; j < 256; ++j) {
+                const int rj = s_qr[j];
+                rank += (rj < rl || (rj == rl && j < l)) ? 1 : 0;
             }
-            const int r2 = min(G.r_cap, 2 * lo + 2);
-            if (nbr_count<true>(G, t, h, w, r2) >= bh) hi = r2;
-            else { lo = min(r2 + 1, G.r_cap); hi = G.r_cap; }
+            s_qp[rank] = l;
         }
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (nbr_count<DISK>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
-        }
-        r = lo;
-        c = nbr_count<DISK>(G, t, h, w, r);
+        __syncthreads();
+        const int l = s_qp[(tile & 1) * 128 + tid];
+        h = trq * G.th + ((l & 127) >> G.tw_log2);
+        w = (tcq - (tile & 1) + (l >> 7)) * G.tw + (l & (G.tw - 1));
+        valid = h < G.H && w < G.W;
+        r = s_qr[l];
+        c = s_qc[l];
+        mask[G.off_group + ((size_t)g * G.nQ + tile) * 128 + tid] = (uint8_t)l;
     }
-    reinterpret_cast<int32_t*>(mask + G.off_radius)[row] = r;
 
     // ---- retained pairs of the tile
     long long cs = c;

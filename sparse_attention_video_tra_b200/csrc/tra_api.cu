@@ -98,7 +98,10 @@ tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtenso
     const int smem = tra::attn_smem_bytes<D>(G.list_cap, G.rte, G.tiles_per_frame);
     if (smem > kMaxSmem) return TRA_ERR_UNSUPPORTED;
     if (!set_smem(kern, smem)) return TRA_ERR_CUDA;
-    kern<<<dim3((G.nQ + 1) / 2, G.G), C::THREADS, smem, st>>>(q, k, v, G, mask, out);
+    // two query tiles per CTA; with radius-sorted groups, the same slot of
+    // frames 2f and 2f + 1
+    const int ctas = G.qsort ? (G.T + 1) / 2 * G.tiles_per_frame : (G.nQ + 1) / 2;
+    kern<<<dim3(ctas, G.G), C::THREADS, smem, st>>>(q, k, v, G, mask, out);
     return launch_status();
 }
 
@@ -180,10 +183,17 @@ extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void
     if (!plan || !Hent || !mask || !aligned(Hent, 4) || !aligned(mask, 256)) return TRA_ERR_INVALID_ARG;
     if (mask_bytes < plan->mask_bytes) return TRA_ERR_WORKSPACE;
     const tra::Geom& G = plan->geom;
-    if (G.disk)
-        tra::radius_mask_kernel<true><<<dim3(G.nQ, G.G), 128, tra::mask_smem_bytes(G.rte, G.nTh), (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
-    else
-        tra::radius_mask_kernel<false><<<dim3(G.nQ, G.G), 128, tra::mask_smem_bytes(G.rte, G.nTh), (cudaStream_t)stream>>>(G, Hent, (uint8_t*)mask);
+    const dim3 grid(G.nQ, G.G);
+    const int smem = tra::mask_smem_bytes(G.rte, G.nTh, G.qsort != 0);   // at most 44.8 KB
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* m = (uint8_t*)mask;
+    if (G.qsort) {
+        if (G.disk) tra::radius_mask_kernel<true, true><<<grid, 128, smem, st>>>(G, Hent, m);
+        else tra::radius_mask_kernel<false, true><<<grid, 128, smem, st>>>(G, Hent, m);
+    } else {
+        if (G.disk) tra::radius_mask_kernel<true, false><<<grid, 128, smem, st>>>(G, Hent, m);
+        else tra::radius_mask_kernel<false, false><<<grid, 128, smem, st>>>(G, Hent, m);
+    }
     return launch_status();
 }
 

@@ -23,12 +23,13 @@ struct Geom {
     int Bmin;
     double a, b;
     double g[TRA_MAX_RT_EFF + 1];    // gamma^delta
-    long long off_radius, off_count, off_pairs, off_list;
+    long long off_radius, off_count, off_pairs, off_list, off_group;
     float scale_log2;                // log2(e) / sqrt(d)
     unsigned long long wait_ns;      // limit of a pipeline wait
     unsigned long long drain_ns;     // limit of the waits that drain in-flight copies
     int natural;                     // q/k/v/out/entropies in natural token order (4-D TMA boxes)
     int disk;                        // spatial test dh^2 + dw^2 <= s^2 instead of the Chebyshev square
+    int qsort;                       // radius-sorted query groups of tile pairs
 };
 
 }  // namespace tra

@@ -48,7 +48,7 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     if (Bmin < 1 || (long long)Bmin > N) return TRA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return TRA_ERR_UNSUPPORTED;
     if (flags & ~(TRA_FLAG_TILE_W_MASK | TRA_FLAG_DEBUG_NO_WAIT | TRA_FLAG_OUT_BF16 | TRA_FLAG_NATURAL |
-                  TRA_FLAG_DISK))
+                  TRA_FLAG_DISK | TRA_FLAG_QSORT))
         return TRA_ERR_INVALID_ARG;
 
     if (H > TRA_MAX_HW || W > TRA_MAX_HW) return TRA_ERR_UNSUPPORTED;
@@ -125,6 +125,10 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     G.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     G.wait_ns = (flags & TRA_FLAG_DEBUG_NO_WAIT) ? 0ull : 2000000000ull;
     G.natural = (flags & TRA_FLAG_NATURAL) ? 1 : 0;
+    // radius-sorted groups pair tiles 2p and 2p+1, which sit side by side in
+    // one tile row only when a frame has an even number of tile columns
+    G.qsort = (flags & TRA_FLAG_QSORT) ? 1 : 0;
+    if (G.qsort && (G.nTw & 1)) return TRA_ERR_UNSUPPORTED;
     G.drain_ns = 2000000000ull;
 
     // mask buffer layout
@@ -133,6 +137,8 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     G.off_count = (long long)off;   off = align256(off + sizeof(int) * (size_t)heads * nQ);
     G.off_pairs = (long long)off;   off = align256(off + sizeof(long long) * (size_t)heads * nQ);
     G.off_list = (long long)off;    off = align256(off + sizeof(uint16_t) * (size_t)heads * nQ * G.list_cap);
+    G.off_group = 0;
+    if (G.qsort) { G.off_group = (long long)off; off = align256(off + (size_t)heads * nQ * 128); }
 
     tra_plan_s* p = new (std::nothrow) tra_plan_s;
     if (!p) return TRA_ERR_INVALID_ARG;
@@ -162,6 +168,7 @@ extern "C" tra_status tra_plan_query(tra_plan plan, tra_plan_info* info)
     info->off_tile_count = (size_t)G.off_count;
     info->off_tile_pairs = (size_t)G.off_pairs;
     info->off_list = (size_t)G.off_list;
+    info->off_group = (size_t)G.off_group;
     return TRA_OK;
 }
 

@@ -35,12 +35,13 @@ class WorkloadRun:
     mask, each with its own V (drawn untimed at setup)."""
 
     def __init__(self, wl: synth.Workload, calls: int = 1, seed_offset: int = 0, device="cuda",
-                 b: float | None = None):
+                 b: float | None = None, flags: int = 0):
         self.wl = wl
         self.calls = calls
+        self.flags = flags
         self.device = device
         T, H, W, G, d = wl.T, wl.H, wl.W, wl.heads, wl.d
-        probe = Plan(T, H, W, G, d, wl.a, 0.0, wl.gamma, wl.Rt, wl.Bmin)
+        probe = Plan(T, H, W, G, d, wl.a, 0.0, wl.gamma, wl.Rt, wl.Bmin, flags)    # sizes every buffer
         self.info = probe.info
         i = self.info
         seed = synth.SEED_BASE + wl.index + 1000 * seed_offset
@@ -66,7 +67,7 @@ class WorkloadRun:
             b = wl.b if wl.b is not None else self.calibrate_b(wl.target_retained)
         probe.close()
         self.b = b
-        self.plan = Plan(T, H, W, G, d, wl.a, b, wl.gamma, wl.Rt, wl.Bmin)
+        self.plan = Plan(T, H, W, G, d, wl.a, b, wl.gamma, wl.Rt, wl.Bmin, flags)
         self.plan.radius_and_mask(self.H, self.mask)
         torch.cuda.synchronize()
         self.retained_pairs = self.pairs()
@@ -74,7 +75,7 @@ class WorkloadRun:
     # ------------------------------------------------------------ calibration
     def retained_fraction(self, b: float) -> float:
         wl = self.wl
-        p = Plan(wl.T, wl.H, wl.W, wl.heads, wl.d, wl.a, b, wl.gamma, wl.Rt, wl.Bmin)
+        p = Plan(wl.T, wl.H, wl.W, wl.heads, wl.d, wl.a, b, wl.gamma, wl.Rt, wl.Bmin, self.flags)
         p.radius_and_mask(self.H, self.mask)
         frac = float(p.mask_views(self.mask)[2].sum().item()) / (wl.heads * float(wl.N) ** 2)
         p.close()

@@ -105,3 +105,48 @@ def test_wan720_full_size_natural_layout_is_bit_identical(run):
     assert torch.equal(a[3][listed], b[3][listed])    # every listed entry, full flags included
     assert torch.equal(gh.to_natural(run.out, i), out)
     plan.close()
+
+
+def test_wan720_full_size_qsort(run):
+    """Radius-sorted query groups (TRA_FLAG_QSORT, the benchmark's default at
+    this shape): radii as without the flag, the group order and sampled group
+    lists equal to the oracle's, sampled outputs within tolerance."""
+    wl, i = run.wl, run.info
+    T, H, W, d, N = wl.T, wl.H, wl.W, wl.d, wl.N
+    plan = _plan(run, tra.TRA_FLAG_QSORT)
+    mask, out = plan.new_mask(), plan.new_out()
+    plan.radius_and_mask(run.H, mask)
+    plan.attention(run.q, run.k, run.v[0], mask, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    rad, cnt, pairs, lst = plan.mask_views(mask)
+    assert torch.equal(rad, run.plan.mask_views(run.mask)[0])
+    rng = np.random.default_rng(13)
+    sel = [0, wl.heads - 1]
+    G = len(sel)
+    nat = gh.tile_major_index(i)
+    r_nat = np.zeros((G, N), np.int32)
+    r_nat[:, nat[nat >= 0]] = rad[sel].cpu().numpy()[:, nat >= 0]
+    r_nat = r_nat.reshape(-1)
+    perm, members = oracle.query_groups(r_nat, G, (T, H, W), (i.tile_h, i.tile_w))
+    np.testing.assert_array_equal(plan.group_view(mask)[sel].cpu().numpy(), perm)
+    Hg = gh.to_natural(run.H[sel], i).cpu().numpy().reshape(G * N)
+    for t in rng.choice(i.n_tiles, size=3, replace=False):
+        for gi, g in enumerate(sel):
+            mem = members[gi * i.n_tiles + int(t)][None]
+            row = oracle.block_mask_sets(r_nat, G, (T, H, W), wl.gamma, wl.Rt, (i.tile_h, i.tile_w), mem)[0]
+            n = int(cnt[g, t])
+            e = lst[g, t, :n].cpu().numpy().view(np.uint16).astype(np.int64)
+            dense = np.zeros(i.n_tiles, np.uint8)
+            dense[e & 0x7FFF] = np.where(e & 0x8000, 3, 1)
+            np.testing.assert_array_equal(dense, row)
+            q = mem[0][mem[0] >= 0]
+            _, c_mem, _ = oracle.radius(Hg[q], G, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, queries=q)
+            assert int(pairs[g, t]) == int(c_mem.sum())
+    bits = lambda x: gh.bf16_bits(gh.to_natural(x[sel], i))     # noqa: E731
+    qb, kb, vb = bits(run.q), bits(run.k), bits(run.v[0])
+    o = gh.to_natural(out[sel], i).float().cpu().numpy().reshape(G * N, d)
+    queries = np.sort(rng.choice(G * N, size=24, replace=False))
+    Oref = oracle.attention(qb, kb, vb, r_nat, G, (T, H, W), d, wl.gamma, wl.Rt, queries=queries)
+    gh.check_attention(o[queries], Oref)
+    plan.close()
