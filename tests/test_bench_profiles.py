@@ -42,3 +42,18 @@ def test_stale_or_missing_summary_reports_no_traffic(tmp_path, monkeypatch):
     (tmp_path / "profiles" / f"{bench.ROOFLINE_KERNEL}_wan720_traffic.txt").write_text(
         f"source_sha256: {bench.source_sha256()}\ndram_bytes_per_launch: 123\n")
     assert bench.recorded_traffic(bench.ROOFLINE_KERNEL, "wan720") == 123.0
+
+
+def test_query_group_default_follows_the_plan():
+    """--qsort auto turns radius-sorted query groups on exactly where the plan
+    accepts them (an even number of tile columns per frame)."""
+    import pytest
+    from sparse_attention_video_tra_b200 import TRA_FLAG_QSORT, TraError, synth
+    W = synth.WORKLOADS
+    assert bench.query_group_flags("auto", W["wan720"]) == TRA_FLAG_QSORT       # 10 tile columns
+    assert bench.query_group_flags("auto", W["hunyuan720"]) == TRA_FLAG_QSORT
+    assert bench.query_group_flags("auto", W["len4x"]) == TRA_FLAG_QSORT
+    assert bench.query_group_flags("auto", W["wan480"]) == 0                    # 13 tile columns
+    assert bench.query_group_flags("off", W["wan720"]) == 0
+    with pytest.raises(TraError):
+        bench.query_group_flags("on", W["wan480"])
