@@ -45,6 +45,10 @@ MUTANTS = [
      [f"{PINS}::test_entropy_q_zero_subsampled_keeps_log_n"]),
     ("attention without the 1/sqrt(d) scale", "double sigma = 1.0 / sqrt((double)d);", "double sigma = 1.0;", 2,
      [f"{PINS}::test_dense_case_equals_sdpa"]),
+    ("set block mask never marks full", "out[set * nK + kb] = (uint8_t)(some && any ? (all ? 3 : 1) : 0);",
+     "out[set * nK + kb] = (uint8_t)(some && any ? 1 : 0);", 1,
+     ["tests/test_oracle_qsort_pins.py::test_sets_equal_tiles_when_sets_are_tiles",
+      "tests/test_oracle_qsort_pins.py::test_sets_equal_bruteforce"]),
     ("calibration cut one key late", "if (cum >= mass) { kk = j + 1; break; }", "if (cum > mass) { kk = j + 2; break; }", 1,
      [f"{CALIB}::test_uniform_attention_needs_ceil_mass_times_n", f"{CALIB}::test_topk_matches_numpy_sort"]),
 ]

@@ -40,11 +40,14 @@ def _tile_members(G, grid, tile):
 def test_sets_equal_tiles_when_sets_are_tiles(grid, tile, metric):
     T, H, W = grid
     G, N = 2, T * H * W
-    r = np.random.default_rng(1).integers(0, 7, G * N).astype(np.int32)
-    mem = _tile_members(G, grid, tile)
-    a = oracle.block_mask_sets(r, G, grid, 0.8, 2, tile, mem, metric=metric)
-    b = oracle.block_mask(r, G, grid, 0.8, 2, tile, tile, metric=metric)
-    np.testing.assert_array_equal(a, b)
+    for lo, hi in ((0, 7), (40, 41)):      # mixed small radii; radii that make every reachable tile full
+        r = np.random.default_rng(1).integers(lo, hi, G * N).astype(np.int32)
+        mem = _tile_members(G, grid, tile)
+        a = oracle.block_mask_sets(r, G, grid, 0.8, 2, tile, mem, metric=metric)
+        b = oracle.block_mask(r, G, grid, 0.8, 2, tile, tile, metric=metric)
+        np.testing.assert_array_equal(a, b)
+        if lo == 40:
+            assert (b == 3).any()
 
 
 @pytest.mark.parametrize("disk", [False, True])
@@ -52,23 +55,27 @@ def test_sets_equal_bruteforce(disk):
     T, H, W, gamma, Rt = 3, 7, 9, 0.8, 1
     N = T * H * W
     rng = np.random.default_rng(2)
-    r = rng.integers(0, 6, N).astype(np.int32)
-    M = bf.token_mask(T, H, W, gamma, Rt, r, disk=disk)        # [N, N] keep
     kt = (2, 4)
     kid, nK = bf.tile_ids(T, H, W, *kt)
-    sets = np.full((6, 10), -1, np.int64)
-    for s in range(6):
-        k = rng.integers(1, 11)
-        sets[s, :k] = rng.choice(N, size=k, replace=False)
-    got = oracle.block_mask_sets(r, 1, (T, H, W), gamma, Rt, kt, sets,
-                                 metric=oracle.DISK if disk else oracle.CHEBYSHEV)
-    for s in range(6):
-        q = sets[s][sets[s] >= 0]
-        for kb in range(nK):
-            keys = np.nonzero(kid == kb)[0]
-            blk = M[np.ix_(q, keys)]
-            want = (3 if blk.all() else 1) if blk.any() else 0
-            assert got[s, kb] == want
+    n_full = 0
+    for lo, hi in ((0, 6), (20, 30)):      # small radii; radii that make full tiles
+        r = rng.integers(lo, hi, N).astype(np.int32)
+        M = bf.token_mask(T, H, W, gamma, Rt, r, disk=disk)        # [N, N] keep
+        sets = np.full((6, 10), -1, np.int64)
+        for s in range(6):
+            k = rng.integers(1, 11)
+            sets[s, :k] = rng.choice(N, size=k, replace=False)
+        got = oracle.block_mask_sets(r, 1, (T, H, W), gamma, Rt, kt, sets,
+                                     metric=oracle.DISK if disk else oracle.CHEBYSHEV)
+        for s in range(6):
+            q = sets[s][sets[s] >= 0]
+            for kb in range(nK):
+                keys = np.nonzero(kid == kb)[0]
+                blk = M[np.ix_(q, keys)]
+                want = (3 if blk.all() else 1) if blk.any() else 0
+                n_full += want == 3
+                assert got[s, kb] == want
+    assert n_full > 0
 
 
 def test_groups_partition_pairs_sorted_by_radius():
