@@ -266,6 +266,26 @@ TRA_API tra_status tra_calibrate_topk(tra_plan plan, const void* q, const void* 
                                       int query_tile_stride, float* H_out, int* k_out, tra_stream stream);
 
 /*
+ * tra_calibrate_fit -- the plan's budget constants from calibration pairs
+ * (the summary's Intuition I: the number of keys a query needs grows
+ * log-linearly with its entropy, B ~ tau * exp(H_i); the fit lets the slope
+ * differ from 1).  Ordinary least squares of ln k_i on H_i,
+ *     ln k = a * H + b,
+ * over the rows with k_i >= 1 and a finite H_i (so the pad rows of
+ * tra_calibrate_topk, NaN / -1, drop out).  The result goes straight into
+ * tra_plan_create(..., a, b, ...).
+ *   H, k       HOST arrays of n rows: fp32 entropies and int32 counts (the
+ *              outputs of tra_calibrate_topk copied to the host, any order)
+ *   a, b       out: slope and intercept
+ *   rows_used  out, may be NULL: the number of rows the fit used
+ * Returns TRA_ERR_INVALID_ARG for a null pointer, n < 0, fewer than two
+ * usable rows, or usable rows that all share one H (a and b are then left
+ * unchanged).  Host arithmetic only (fp64); no CUDA call.
+ */
+TRA_API tra_status tra_calibrate_fit(const float* H, const int32_t* k, long long n, double* a, double* b,
+                                     long long* rows_used);
+
+/*
  * tra_plan_status -- read and clear the current device's error word.  Call
  * after synchronising the streams that ran this library's kernels.  Returns
  * TRA_OK, TRA_ERR_TIMEOUT or TRA_ERR_DEVICE_CHECK (or TRA_ERR_CUDA if the

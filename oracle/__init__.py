@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
             [ctypes.c_double, ctypes.c_int, ctypes.c_int, _I64P, ctypes.c_int64, _F64P]
         L.oracle_topk_count.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 5 + \
             [ctypes.c_double, _I64P, ctypes.c_int64, _I64P]
+        L.oracle_fit_log_linear.argtypes = [_F64P, _I64P, ctypes.c_int64, _F64P, _F64P, _F64P]
+        L.oracle_fit_log_linear.restype = ctypes.c_int64
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -285,6 +287,21 @@ def topk_count(q, k, G, grid, d, mass, queries=None) -> np.ndarray:
     lib().oracle_topk_count(qa.ctypes.data, ka.ctypes.data, tq, G, T, H, W, d, float(mass), qp, nq,
                             _ptr(out, _I64P))
     return out
+
+
+def fit_log_linear(H, k):
+    """Calibration fit: least squares of ln k = a*H + b over the rows with
+    k >= 1 and a finite H.  Returns (a, b, r2, rows used); raises ValueError
+    when fewer than two usable rows remain or their H are all equal."""
+    Hd = np.ascontiguousarray(np.asarray(H, dtype=np.float64).reshape(-1))
+    kd = np.ascontiguousarray(np.asarray(k, dtype=np.int64).reshape(-1))
+    assert Hd.size == kd.size
+    a, b, r2 = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    m = lib().oracle_fit_log_linear(_ptr(Hd, _F64P), _ptr(kd, _I64P), Hd.size,
+                                    ctypes.byref(a), ctypes.byref(b), ctypes.byref(r2))
+    if m < 0:
+        raise ValueError("fewer than two usable (H, k) rows, or all H equal")
+    return a.value, b.value, r2.value, int(m)
 
 
 def num_threads() -> int:

@@ -489,6 +489,48 @@ void oracle_topk_count(const void* q, const void* k, int type, int G, int T, int
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Calibration fit ([TRA] Intuition I: the number of keys a query needs      */
+/* grows log-linearly with its entropy, B ~ tau*exp(H_i), i.e. ln B is       */
+/* linear in H with slope 1 and intercept ln tau; the fit generalises the    */
+/* slope to a).  Ordinary least squares of y = ln k_i on x = H_i,            */
+/*   ln k = a*H + b,                                                         */
+/* over the rows with k_i >= 1 and a finite H_i, in two passes: the means,   */
+/* then the centred sums  a = S_xy / S_xx,  b = mean(y) - a*mean(x).         */
+/* r2_out (optional) = S_xy^2 / (S_xx * S_yy), the share of the variance of  */
+/* ln k the line explains.  Returns the number of rows used, or -1 (nothing  */
+/* written) when fewer than two rows are usable or their H are all equal.    */
+/* ------------------------------------------------------------------------ */
+static double fit_y(int64_t k) { return log((double)k); }
+
+int64_t oracle_fit_log_linear(const double* H, const int64_t* k, int64_t n,
+                              double* a_out, double* b_out, double* r2_out)
+{
+    int64_t m = 0;
+    double sx = 0.0, sy = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        if (k[i] < 1 || !isfinite(H[i])) continue;
+        ++m;
+        sx += H[i];
+        sy += fit_y(k[i]);
+    }
+    if (m < 2) return -1;
+    double mx = sx / (double)m, my = sy / (double)m;
+    double sxx = 0.0, sxy = 0.0, syy = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        if (k[i] < 1 || !isfinite(H[i])) continue;
+        double dx = H[i] - mx, dy = fit_y(k[i]) - my;
+        sxx += dx * dx;
+        sxy += dx * dy;
+        syy += dy * dy;
+    }
+    if (!(sxx > 0.0)) return -1;
+    *a_out = sxy / sxx;
+    *b_out = my - *a_out * mx;
+    if (r2_out) *r2_out = syy > 0.0 ? (sxy * sxy) / (sxx * syy) : 1.0;
+    return m;
+}
+
 /* threads the OpenMP runtime will use (for the reported CPU baseline) */
 int oracle_num_threads(void)
 {

@@ -20,7 +20,8 @@ from dataclasses import dataclass
 __all__ = [
     "TraError", "PlanInfo", "Plan", "library_path", "load_library",
     "tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
-    "tra_radius_and_mask", "tra_attention", "tra_calibrate_topk", "tra_plan_status", "tra_status_string",
+    "tra_radius_and_mask", "tra_attention", "tra_calibrate_topk", "tra_calibrate_fit", "tra_plan_status",
+    "tra_status_string",
     "TRA_FLAG_DEBUG_NO_WAIT", "TRA_FLAG_OUT_BF16", "TRA_FLAG_NATURAL", "TRA_FLAG_DISK", "TRA_FLAG_QSORT",
     "tra_flag_tile_w",
 ]
@@ -113,6 +114,9 @@ def load_library() -> ctypes.CDLL:
     L.tra_attention.restype = st
     L.tra_calibrate_topk.argtypes = [vp, vp, vp, ctypes.c_double, i, vp, vp, vp]
     L.tra_calibrate_topk.restype = st
+    L.tra_calibrate_fit.argtypes = [vp, vp, ctypes.c_longlong, ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+    L.tra_calibrate_fit.restype = st
     L.tra_plan_status.argtypes = [vp]
     L.tra_plan_status.restype = st
     L.tra_status_string.argtypes = [st]
@@ -171,6 +175,14 @@ def tra_calibrate_topk(plan, q_ptr, k_ptr, mass, query_tile_stride, H_ptr, k_out
     _check("tra_calibrate_topk", load_library().tra_calibrate_topk(plan, q_ptr, k_ptr, float(mass),
                                                                    int(query_tile_stride), H_ptr, k_out_ptr,
                                                                    stream))
+
+
+def tra_calibrate_fit(H_ptr, k_ptr, n) -> tuple[float, float, int]:
+    """(a, b, rows used) of ln k = a*H + b from n host rows (fp32 H, int32 k)."""
+    a, b, m = ctypes.c_double(), ctypes.c_double(), ctypes.c_longlong()
+    _check("tra_calibrate_fit", load_library().tra_calibrate_fit(H_ptr, k_ptr, int(n), ctypes.byref(a),
+                                                                 ctypes.byref(b), ctypes.byref(m)))
+    return a.value, b.value, m.value
 
 
 def tra_plan_status(plan) -> int:

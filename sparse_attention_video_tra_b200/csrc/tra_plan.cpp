@@ -172,6 +172,34 @@ extern "C" tra_status tra_plan_query(tra_plan plan, tra_plan_info* info)
     return TRA_OK;
 }
 
+// Least squares of ln k on H in one pass over the rows (running means and
+// co-moments, updated row by row so no second pass or large sums are needed):
+// with dx = x - mean_x before the row and mean_y after it,
+// C_xx += dx * (x - mean_x'), C_xy += dx * (y - mean_y').
+extern "C" tra_status tra_calibrate_fit(const float* H, const int32_t* k, long long n, double* a, double* b,
+                                        long long* rows_used)
+{
+    if (!H || !k || !a || !b || n < 0) return TRA_ERR_INVALID_ARG;
+    long long m = 0;
+    double mean_x = 0.0, mean_y = 0.0, cxx = 0.0, cxy = 0.0;
+    for (long long i = 0; i < n; ++i) {
+        const double x = (double)H[i];
+        if (k[i] < 1 || !std::isfinite(x)) continue;
+        const double y = std::log((double)k[i]);
+        ++m;
+        const double dx = x - mean_x;
+        mean_x += dx / (double)m;
+        mean_y += (y - mean_y) / (double)m;
+        cxx += dx * (x - mean_x);
+        cxy += dx * (y - mean_y);
+    }
+    if (rows_used) *rows_used = m;
+    if (m < 2 || !(cxx > 0.0)) return TRA_ERR_INVALID_ARG;
+    *a = cxy / cxx;
+    *b = mean_y - *a * mean_x;
+    return TRA_OK;
+}
+
 extern "C" const char* tra_status_string(tra_status s)
 {
     switch (s) {

@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = set(declared_functions())
     assert {"tra_plan_create", "tra_plan_destroy", "tra_plan_query", "tra_permute", "tra_entropy",
-            "tra_radius_and_mask", "tra_attention", "tra_plan_status", "tra_status_string"} <= names
+            "tra_radius_and_mask", "tra_attention", "tra_calibrate_topk", "tra_calibrate_fit",
+            "tra_plan_status", "tra_status_string"} <= names
 
 
 def test_library_exports_every_declared_symbol():
@@ -76,7 +77,7 @@ def test_natural_layout_flag():
     assert not q.natural and q.io_rows == q.info.N_pad
     assert p.info == q.info                      # same geometry and mask layout
     with pytest.raises(tra.TraError):
-        tra.tra_plan_create(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=1 << 20)
+        tra.tra_plan_create(4, 8, 8, 2, 64, 1.0, 0.0, 0.7, 2, 8, flags=1 << 21)   # no such flag
 
 
 @pytest.mark.parametrize("grid,gamma,Rt", [((21, 45, 80), 0.8, 6), ((4, 8, 8), 0.7, 2), ((3, 7, 9), 0.5, 1),

@@ -5,7 +5,11 @@ gist.science summary, section 2, Intuition I: the key density a query needs
 follows its entropy).
 
 Closed forms (uniform attention; one dominant key among equal others), the
-independent numpy sort in tests/bruteforce.py, and monotonicity in the mass."""
+independent numpy sort in tests/bruteforce.py, and monotonicity in the mass.
+
+The fit ln k = a*H + b that turns those pairs into the plan's budget
+constants is pinned by a hand-worked three-point case, the line through two
+points, exact recovery of a known (a, b), and numpy.polyfit on noisy data."""
 import math
 
 import numpy as np
@@ -69,3 +73,62 @@ def test_topk_monotone_in_mass_and_bounded():
         cur = oracle.topk_count(q, k, 1, (T, H, W), d, mass)
         assert np.all(cur >= prev) and np.all((1 <= cur) & (cur <= N))
         prev = cur
+
+
+# ---------------------------------------------------------------- the fit ln k = a*H + b
+def test_fit_hand_worked_three_points():
+    """x = H = (0, 1, 2), k = (1, 2, 8): y = ln k = (0, 1, 3)*ln 2.  By hand:
+    mean x = 1, mean y = (4/3) ln 2, S_xy = 3 ln 2, S_xx = 2, so
+    a = (3/2) ln 2 and b = (4/3 - 3/2) ln 2 = -(1/6) ln 2; S_yy = (42/9) ln^2 2,
+    r2 = 9 ln^2 2 / (2 * 42/9 ln^2 2) = 81/84."""
+    a, b, r2, m = oracle.fit_log_linear([0.0, 1.0, 2.0], [1, 2, 8])
+    L2 = math.log(2.0)
+    assert m == 3
+    assert a == pytest.approx(1.5 * L2, rel=1e-14)
+    assert b == pytest.approx(-L2 / 6.0, rel=1e-13)
+    assert r2 == pytest.approx(81.0 / 84.0, rel=1e-14)
+
+
+def test_fit_two_points_is_the_line_through_them():
+    H1, H2, k1, k2 = 1.25, 4.0, 3, 170
+    a, b, r2, m = oracle.fit_log_linear([H1, H2], [k1, k2])
+    slope = (math.log(k2) - math.log(k1)) / (H2 - H1)
+    assert a == pytest.approx(slope, rel=1e-14)
+    assert b == pytest.approx(math.log(k1) - slope * H1, rel=1e-13, abs=1e-14)
+    assert r2 == pytest.approx(1.0, rel=1e-14)
+
+
+def test_fit_recovers_exact_log_linear_data():
+    """H_i placed exactly on ln k = 1.3*H - 0.5 for integer k_i (the tau*exp(H)
+    law with slope 1.3): the fit returns (1.3, -0.5)."""
+    rng = np.random.default_rng(11)
+    k = rng.integers(1, 5000, 400)
+    H = (np.log(k) + 0.5) / 1.3
+    a, b, r2, m = oracle.fit_log_linear(H, k)
+    assert m == 400
+    assert a == pytest.approx(1.3, abs=1e-12)
+    assert b == pytest.approx(-0.5, abs=1e-11)
+    assert r2 == pytest.approx(1.0, abs=1e-12)
+
+
+def test_fit_matches_numpy_polyfit_on_noisy_data():
+    """Against an independent least-squares routine (numpy.polyfit, degree 1)."""
+    rng = np.random.default_rng(12)
+    H = rng.uniform(2.0, 10.0, 3000)
+    k = np.maximum(1, np.round(np.exp(0.9 * H + 0.7 + rng.normal(0, 0.6, H.size)))).astype(np.int64)
+    a, b, r2, m = oracle.fit_log_linear(H, k)
+    pa, pb = np.polyfit(H, np.log(k), 1)
+    assert a == pytest.approx(pa, rel=1e-10)
+    assert b == pytest.approx(pb, rel=1e-10, abs=1e-10)
+    assert 0.5 < r2 < 1.0
+
+
+def test_fit_ignores_unusable_rows_and_rejects_degenerate_input():
+    H = [0.0, 1.0, 2.0, float("nan"), 5.0, float("inf")]
+    k = [1, 2, 8, 40, 0, 7]          # the NaN-H, k=0 and inf-H rows are not used
+    a, b, r2, m = oracle.fit_log_linear(H, k)
+    assert m == 3 and a == pytest.approx(1.5 * math.log(2.0), rel=1e-14)
+    with pytest.raises(ValueError):
+        oracle.fit_log_linear([1.0, 2.0], [5, -1])          # one usable row
+    with pytest.raises(ValueError):
+        oracle.fit_log_linear([3.0, 3.0, 3.0], [1, 5, 9])   # no spread in H

@@ -51,6 +51,14 @@ MUTANTS = [
       "tests/test_oracle_qsort_pins.py::test_sets_equal_bruteforce"]),
     ("calibration cut one key late", "if (cum >= mass) { kk = j + 1; break; }", "if (cum > mass) { kk = j + 2; break; }", 1,
      [f"{CALIB}::test_uniform_attention_needs_ceil_mass_times_n", f"{CALIB}::test_topk_matches_numpy_sort"]),
+    ("calibration fit through the origin (no intercept)", "double dx = H[i] - mx, dy = fit_y(k[i]) - my;",
+     "double dx = H[i], dy = fit_y(k[i]);", 1,
+     [f"{CALIB}::test_fit_hand_worked_three_points", f"{CALIB}::test_fit_matches_numpy_polyfit_on_noisy_data"]),
+    ("calibration fit in log2", "static double fit_y(int64_t k) { return log((double)k); }",
+     "static double fit_y(int64_t k) { return log2((double)k); }", 1,
+     [f"{CALIB}::test_fit_hand_worked_three_points", f"{CALIB}::test_fit_recovers_exact_log_linear_data"]),
+    ("calibration fit regresses H on ln k", "*a_out = sxy / sxx;", "*a_out = syy / sxy;", 1,
+     [f"{CALIB}::test_fit_hand_worked_three_points", f"{CALIB}::test_fit_matches_numpy_polyfit_on_noisy_data"]),
 ]
 
 
