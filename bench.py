@@ -2,6 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan720] [--impl tra|reference]
 
+With --gpus N > 1 and no torchrun environment, the script starts N ranks of
+itself through torch.distributed.run on this node (one per GPU); under
+torchrun it checks that WORLD_SIZE equals N.
+
 A step is one pass of the whole hot path over one batch of synthetic input:
 dense (or key-subsampled) warm-up entropy, one radius/mask build, then
 `calls` attention calls that reuse the mask with a fresh V each (10 for the
@@ -30,6 +34,9 @@ import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+# B200 exponential unit (MUFU ex2): 16 results per clock per SM, 148 SMs, at
+# the 1965 MHz maximum SM clock -- the bound of the entropy kernel
+MUFU_EX2_PER_S = 16 * 148 * 1965e6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "TRA attention retained-pair TFLOP/s (bf16) at 21x45x80 tokens, 40 heads; ms/call reported"
 
@@ -43,20 +50,38 @@ def peaks():
 
 
 # ---------------------------------------------------------------- distributed
-def dist_setup():
+def dist_setup(expected_world: int = 0):
+    """Rank and world size from the torchrun environment; one process per GPU
+    (LOCAL_RANK picks the device).  NCCL when GPUs are present, else gloo
+    (the CPU tests).  The process group gets a short timeout so that ranks
+    waiting on a rank that died end with an error instead of hanging."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if expected_world and world != expected_world:
+        raise SystemExit(f"bench.py: --gpus {expected_world} but WORLD_SIZE={world}")
+    if torch.cuda.is_available():
+        if local >= torch.cuda.device_count():
+            raise SystemExit(f"bench.py: LOCAL_RANK {local} but only {torch.cuda.device_count()} GPUs are visible")
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
         backend = "nccl" if torch.cuda.is_available() else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
     return rank, world
+
+
+def relaunch(argv, n: int) -> int:
+    """Start n ranks of this script on this node through torch.distributed.run
+    (rendezvous on 127.0.0.1, a free port); returns their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def max_over_ranks(x: float, world: int) -> float:
@@ -281,16 +306,68 @@ def _oracle_entropy_tiled(oracle, qb, kb, G, wl, idx):
     return oracle.entropy(qb, kb, G, (wl.T, wl.H, wl.W), wl.d, key_stride=wl.key_stride, ktile=(th, tw), queries=idx)
 
 
+# ---------------------------------------------------------------- workload and config (both arms)
+def bench_workload(args, rank: int, world: int):
+    """The workload this rank runs: the named one, with the command line's
+    head count, retained fraction or b; with --shard heads only this rank's
+    contiguous slice of the heads.  Returns (workload, all heads, the rank's
+    (first head, count)).  Host-side only (no GPU)."""
+    import dataclasses
+    sys.path.insert(0, ROOT)
+    from sparse_attention_video_tra_b200 import synth
+    from sparse_attention_video_tra_b200.runner import shard_heads
+    wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        wl = dataclasses.replace(wl, heads=args.heads, name=wl.name.replace(f"{wl.heads} heads", f"{args.heads} heads"))
+    if args.retained:
+        wl = dataclasses.replace(wl, target_retained=float(args.retained), b=None)
+    if args.b is not None:
+        wl = dataclasses.replace(wl, b=float(args.b))
+    total = wl.heads
+    first, count = 0, wl.heads
+    if args.shard == "heads":
+        first, count = shard_heads(wl.heads, world, rank)
+        if count == 0:
+            raise SystemExit(f"rank {rank}: no heads left to shard ({wl.heads} heads over {world} ranks)")
+        wl = dataclasses.replace(wl, heads=count)
+    return wl, total, (first, count)
+
+
+def attention_calls(args) -> int:
+    return args.calls if args.calls else (10 if args.workload == "wan720" else 1)
+
+
+def bench_config(args, wl, total_heads: int, world: int, b: float) -> dict:
+    """The `config` object of the JSON line, the same for both arms: the
+    workload, the batch, the plan's parameters and tile choice."""
+    from sparse_attention_video_tra_b200 import Plan
+    sharded = args.shard == "heads"
+    flags = query_group_flags(args.qsort, wl)
+    p = Plan(wl.T, wl.H, wl.W, 1, wl.d, wl.a, b, wl.gamma, wl.Rt, wl.Bmin, flags)
+    tile_desc = f"1x{p.info.tile_h}x{p.info.tile_w}"
+    p.close()
+    return {"workload": args.workload_name if hasattr(args, "workload_name") else wl.name,
+            "global_batch": total_heads if sharded else total_heads * max(world, 1), "seq_len": wl.N,
+            "parallelism": (f"heads sharded over {world} GPUs, no collective on the path" if sharded
+                            else f"independent head-batch replicas x{world}"),
+            "attention_calls_per_step": attention_calls(args),
+            "a": wl.a, "b": round(float(b), 6), "gamma": wl.gamma, "Rt": wl.Rt, "Bmin": wl.Bmin,
+            "tile": tile_desc,
+            "query_groups": "radius-sorted groups (TRA_FLAG_QSORT)" if flags else "spatial tiles",
+            "inputs": "resident in HBM, larger than L2; L2 flushed before every step"}
+
+
 # ---------------------------------------------------------------- arms
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
     sys.path.insert(0, ROOT)
-    from sparse_attention_video_tra_b200 import synth
     import oracle
-    wl = synth.WORKLOADS[args.workload]
+    wl, total_heads, _ = bench_workload(args, 0, 1)
+    args.workload_name = synth_name(args, total_heads)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    # b for the target retained fraction, found with the oracle on a query sample
+    # b: the workload's fixed value (the one the GPU arm uses); only a
+    # target-fraction run finds its own, with the oracle on a query sample
     b = wl.b
     if b is None:
         b = _oracle_calibrate_b(oracle, wl, dev)
@@ -302,15 +379,26 @@ def run_reference(args, rank, world):
             vals.append((v, desc))
     value = float(np.mean([v for v, _ in vals]))
     desc = vals[-1][1]
+    config = bench_config(args, wl, total_heads, world, b)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "b": b, "sample": "random queries of head 0, whole oracle path"},
+            "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config,
+            "sample": "random queries of head 0, whole oracle path (entropy, radius, attention)",
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": desc["threads"], "kind": "oracle",
                              "sample": f"{desc['queries']} queries of head 0 per step, entropy+radius+attention"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if args.shard == "heads":
+        from sparse_attention_video_tra_b200.runner import shard_heads
+        line["head_slices"] = [list(shard_heads(total_heads, world, r)) for r in range(world)]
     print(json.dumps(line), flush=True)
     return 0
+
+
+def synth_name(args, total_heads: int) -> str:
+    from sparse_attention_video_tra_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    return wl.name.replace(f"{wl.heads} heads", f"{total_heads} heads")
 
 
 def _oracle_calibrate_b(oracle, wl, dev):
@@ -355,25 +443,11 @@ def query_group_flags(mode: str, wl) -> int:
 
 def run_tra(args, rank, world):
     sys.path.insert(0, ROOT)
-    from sparse_attention_video_tra_b200 import Plan, synth
     from sparse_attention_video_tra_b200.runner import WorkloadRun
-    wl = synth.WORKLOADS[args.workload]
-    if args.heads:
-        import dataclasses
-        wl = dataclasses.replace(wl, heads=args.heads, name=wl.name.replace(f"{wl.heads} heads", f"{args.heads} heads"))
-    if args.retained:
-        import dataclasses
-        wl = dataclasses.replace(wl, target_retained=float(args.retained), b=None)
-    calls = args.calls if args.calls else (10 if args.workload == "wan720" else 1)
-    total_heads, workload_name = wl.heads, wl.name
-    if args.shard == "heads":
-        # strong scaling: this rank's contiguous slice of the heads
-        import dataclasses
-        from sparse_attention_video_tra_b200.runner import shard_heads
-        first, count = shard_heads(wl.heads, world, rank)
-        if count == 0:
-            raise SystemExit(f"rank {rank}: no heads left to shard ({wl.heads} heads over {world} ranks)")
-        wl = dataclasses.replace(wl, heads=count)
+    # strong scaling (--shard heads): this rank's contiguous slice of the heads
+    wl, total_heads, _ = bench_workload(args, rank, world)
+    args.workload_name = synth_name(args, total_heads)
+    calls = attention_calls(args)
     flags = query_group_flags(args.qsort, wl)
     run = WorkloadRun(wl, calls=calls, seed_offset=rank, flags=flags)
     dev_idx = torch.cuda.current_device()
@@ -409,10 +483,12 @@ def run_tra(args, rank, world):
     call_ms = [e[2 + c].elapsed_time(e[3 + c]) for e in evs for c in range(calls)]
     attn_s = sum(call_ms) / 1000.0
     flops = run.attention_flops()
+    # value: all timed calls over their summed device time (the whole-job
+    # rate); the per-phase figures below are medians over steps / calls
     value = aggregate(flops * calls * args.steps, attn_s, world) / 1e12
     step_s = sum(step_ms) / 1000.0
     step_tflops = aggregate(flops * calls * args.steps, step_s, world) / 1e12
-    ms_per_step = max_over_ranks(float(np.mean(step_ms)), world)
+    ms_per_step = max_over_ranks(float(np.median(step_ms)), world)
 
     # separate L2-flushed timing of the mask build (its inputs fit in L2)
     mask_runs = []
@@ -427,7 +503,7 @@ def run_tra(args, rank, world):
     mask_cold_ms = float(np.median(mask_runs))
 
     pk, pk_kind = peaks()
-    avg_call_s = attn_s / (calls * args.steps)
+    avg_call_s = float(np.median(call_ms)) / 1000.0
     achieved = flops / avg_call_s / 1e12
     peak = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     computed = run.computed_pairs()
@@ -440,11 +516,23 @@ def run_tra(args, rank, world):
                 "tile_efficiency": round(run.retained_pairs / computed, 4),
                 "frac_of_burst": round(achieved / float(pk.get("bf16_tflops", 1590.0)), 4)}
     mask_bytes_alg = mask_algorithmic_bytes(run)
-    phases = {"entropy_ms": round(float(np.mean(ent_ms)), 3), "mask_ms": round(float(np.mean(mask_ms)), 4),
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ent_s = float(np.median(ent_ms)) / 1000.0
+    ent_rate = run.entropy_pairs() / ent_s
+    ent_bytes = entropy_algorithmic_bytes(run)
+    phases = {"statistic": "median over steps (attention: over calls)",
+              "entropy_ms": round(ent_s * 1000.0, 3), "mask_ms": round(float(np.median(mask_ms)), 4),
               "mask_ms_l2_flushed": round(mask_cold_ms, 4),
-              "mask_hbm_frac": round(mask_bytes_alg / (mask_cold_ms / 1000.0) / 1e9 / float(pk.get("hbm_gbs", 6650.0)), 4),
-              "attention_ms_per_call": round(float(np.mean(call_ms)), 3),
-              "entropy_scores_per_s": run.entropy_pairs() / (float(np.mean(ent_ms)) / 1000.0)}
+              "mask_gbs": round(mask_bytes_alg / (mask_cold_ms / 1000.0) / 1e9, 2),
+              "mask_hbm_frac": round(mask_bytes_alg / (mask_cold_ms / 1000.0) / 1e9 / hbm, 4),
+              "attention_ms_per_call": round(avg_call_s * 1000.0, 3),
+              "entropy_scores_per_s": ent_rate,
+              "entropy_roofline": {"bound": "alu", "unit": "exponentials/s", "achieved": ent_rate,
+                                   "peak": MUFU_EX2_PER_S, "frac": round(ent_rate / MUFU_EX2_PER_S, 4),
+                                   "peak_derivation": "one ex2 per scored pair; MUFU 16/clk/SM x 148 SMs x 1965 MHz",
+                                   "dram_gbs": round(ent_bytes / ent_s / 1e9, 2),
+                                   "dram_frac": round(ent_bytes / ent_s / 1e9 / hbm, 5),
+                                   "algorithmic_bytes": ent_bytes}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -456,27 +544,25 @@ def run_tra(args, rank, world):
 
     e2e = None if args.no_e2e else run_e2e(run, wl, calls, args, world)
     b_used, retained = run.b, run.retained_fraction_now()
-    tile_desc = f"1x{run.info.tile_h}x{run.info.tile_w}"
-    groups_desc = "radius-sorted pairs (TRA_FLAG_QSORT)" if run.plan.qsort else "spatial tiles"
     del run
     sharded = args.shard == "heads"
     line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
             "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
             "dtype": "bf16",
-            "data": "synthetic (seeded Q,K,V with Wan-720p attention shapes; no model weights)",
-            "config": {"workload": workload_name,
-                       "global_batch": total_heads if sharded else wl.heads * world, "seq_len": wl.N,
-                       "parallelism": (f"heads sharded over {world} GPUs, no collective on the path" if sharded
-                                       else f"independent head-batch replicas x{world}"),
-                       "attention_calls_per_step": calls,
-                       "a": wl.a, "b": round(b_used, 6), "gamma": wl.gamma, "Rt": wl.Rt, "Bmin": wl.Bmin,
-                       "tile": tile_desc, "query_groups": groups_desc,
-                       "inputs": "resident in HBM, 774 MB per tensor (> L2); L2 flushed before every step"},
+            "data": "synthetic (seeded Q,K,V with the video-DiT attention shapes; no model weights)",
+            "config": bench_config(args, wl, total_heads, world, b_used),
             "retained_fraction": round(retained, 5), "phases": phases, "step_tflops": round(step_tflops, 3),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": (2 + calls) * args.steps, "clocks": clk, "wall_s_timed": round(t_wall, 3)}
     return line
+
+
+def entropy_algorithmic_bytes(run) -> float:
+    """Bytes the entropy pass must move: Q and K once (bf16, the plan's rows)
+    and one fp32 entropy per row."""
+    i = run.info
+    return i.heads * i.N_pad * (2.0 * i.d * 2 + 4.0)
 
 
 def mask_algorithmic_bytes(run) -> float:
@@ -604,6 +690,7 @@ def main(argv=None):
                          "heads: the workload's heads are split over the ranks (strong scaling)")
     ap.add_argument("--retained", type=float, default=0.0,
                     help="target retained fraction for calibrating b (0 = the workload's own)")
+    ap.add_argument("--b", type=float, default=None, help="budget offset b (default: the workload's)")
     ap.add_argument("--qsort", default="auto", choices=["auto", "on", "off"],
                     help="radius-sorted query groups (TRA_FLAG_QSORT): auto = when the frame has an even "
                          "number of tile columns")
@@ -612,10 +699,13 @@ def main(argv=None):
                     help="head chunks of the end-to-end leg (each its own plan; copies overlap the other chunks)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
-    args = ap.parse_args(argv)
+    raw = list(sys.argv[1:] if argv is None else argv)
+    args = ap.parse_args(raw)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
-    rank, world = dist_setup()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(raw, args.gpus)
+    rank, world = dist_setup(args.gpus if "WORLD_SIZE" in os.environ else 0)
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)

@@ -61,8 +61,11 @@ WORKLOADS = {
     "tiny": Workload("tiny 4x8x8, 2 heads, d=64", 4, 8, 8, 2, 64, 0.7, 2, 8, a=1.0, b=0.0, index=0),
     "wan480": Workload("Wan-1.3B-480p 21x30x52, 12 heads, d=128", 21, 30, 52, 12, 128, 0.8, 6, 8,
                        target_retained=0.15, index=1),
+    # b fixed at the value whose radii keep 15.0 % of all token pairs on this
+    # workload's seeded inputs (found once by bisection on the GPU entropies;
+    # fixed so every run and both benchmark arms use the same plan)
     "wan720": Workload("Wan-14B-720p 21x45x80, 40 heads, d=128", 21, 45, 80, 40, 128, 0.8, 6, 8,
-                       target_retained=0.15, index=2),
+                       b=-1.1450672149658203, target_retained=0.15, index=2),
     "hunyuan720": Workload("HunyuanVideo-720p 33x45x80, 24 heads, d=128, every 8th key tile", 33, 45, 80,
                            24, 128, 0.8, 6, 8, target_retained=0.15, key_stride=8, index=3),
     "len4x": Workload("4x-length 132x45x80, 24 heads, d=128, every 8th key tile", 132, 45, 80, 24, 128,

@@ -84,3 +84,68 @@ def test_shard_heads_partitions_the_heads(heads, world):
     assert max(sizes) - min(sizes) <= 1
     with pytest.raises(ValueError):
         shard_heads(heads, world, world)
+
+
+def _plan_worker(rank, world, port, out):
+    """--shard heads: each rank's workload slice and the plan it builds for it
+    (host side only), gathered over the gloo group."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    from sparse_attention_video_tra_b200 import Plan
+    try:
+        args = bench.main.__globals__["argparse"].Namespace(
+            workload="wan720", heads=0, retained=0.0, b=None, shard="heads", qsort="auto", gpus=world, calls=0)
+        wl, total, (first, count) = bench.bench_workload(args, rank, world)
+        p = Plan(wl.T, wl.H, wl.W, wl.heads, wl.d, wl.a, wl.b, wl.gamma, wl.Rt, wl.Bmin,
+                 bench.query_group_flags("auto", wl))
+        row = torch.tensor([first, count, p.info.heads, total], dtype=torch.int64)
+        rows = [torch.zeros(4, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(rows, row)
+        out.put((rank, [r.tolist() for r in rows]))
+        p.close()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_plans_partition_the_heads():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_plan_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = [q.get(timeout=10) for _ in range(2)]
+    for _, rows in res:
+        assert rows == res[0][1]                      # every rank sees the same table
+        covered = []
+        for first, count, plan_heads, total in rows:
+            assert plan_heads == count > 0 and total == 40
+            covered += list(range(first, first + count))
+        assert sorted(covered) == list(range(40))     # disjoint and complete
+
+
+def test_bench_gpus_2_starts_two_ranks():
+    """`bench.py --gpus 2` outside torchrun starts 2 ranks itself (gloo here);
+    the reference arm runs on rank 0 only and reports the head slices."""
+    import json
+    import subprocess
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    p = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--impl", "reference", "--workload", "tiny",
+                        "--shard", "heads", "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-3000:]
+    lines = [json.loads(x) for x in p.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1                            # rank 0 alone prints
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["scaling"] == "strong"
+    assert line["head_slices"] == [[0, 1], [1, 1]]
+    assert line["config"]["global_batch"] == 2 and line["value"] > 0
