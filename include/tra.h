@@ -40,8 +40,9 @@
  *
  * Errors.  Host-side validation is synchronous and returns a status.  Kernel
  * launches are asynchronous: a failed launch returns TRA_ERR_CUDA.  Faults a
- * kernel detects itself (a bounded wait that gave up, a bad index in a
- * checked build) are recorded in a per-device error word and reported by
+ * kernel detects itself (a bounded wait that gave up; a mask buffer whose
+ * tile counts or listed key tiles are out of range) are recorded in a
+ * per-device error word and reported by
  * tra_plan_status() after the caller synchronises the stream.  On any error
  * the outputs are unspecified.
  *
@@ -222,7 +223,10 @@ TRA_API tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void* m
 
 /*
  * tra_attention -- block-sparse attention with exact token masking
- * (O_i = sum over the retained keys j of softmax(q_i.k_j/sqrt d) v_j).
+ * (O_i = sum over the retained keys j of softmax(q_i.k_j/sqrt d) v_j):
+ * "Token Radius Attention for Efficient Video Generation", section 2,
+ * "Execution Efficace" (attention runs on the query-key blocks the radius
+ * mask keeps) and "Budget-vers-Rayon" (the token mask itself).
  * Inactive key tiles are skipped; inside listed tiles every token pair is
  * tested, so the result equals dense attention under the token mask.  QK^T
  * and PV run on the tensor cores in bf16 with fp32 accumulation; P is

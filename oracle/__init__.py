@@ -40,7 +40,7 @@ def compile_source(src: str, out: str) -> str:
     """gcc the oracle's C source `src` into the shared library `out`."""
     tmp = out + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, src, "-lm"]
+           "-std=gnu11", "-Wall", "-shared", "-fPIC", "-o", tmp, src, "-lquadmath", "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
     return out

@@ -38,14 +38,16 @@
  *     count then sums, row by row, the clipped width 2*isqrt(s^2 - dh^2) + 1,
  *     and r_cap is the smallest r with s(r, Rt')^2 >= (H-1)^2 + (W-1)^2.
  *
- * Build:  gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
- * (fp-contract=off keeps r*g and +1e-9 as two separately rounded operations).
+ * Build:  gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC ... -lquadmath
+ * (fp-contract=off keeps r*g and +1e-9 as two separately rounded operations;
+ * libquadmath gives the budget's exponential in binary128).
  *
  * Layout of every per-token array: [heads][N][...] in natural order.
  * Element arrays are passed as `const void*` with a type flag: 0 = float32,
  * 1 = bfloat16 bit patterns (uint16), 2 = float64.  All arithmetic is fp64.
  */
 #include <math.h>
+#include <quadmath.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -168,14 +170,25 @@ int64_t oracle_count(int T, int H, int W, double gamma, int Rt,
 }
 
 /* E3: token budget from entropy ([TRA] Intuition I).  Hent is the fp32
-   entropy promoted to fp64; a*H and +b are rounded separately. */
+   entropy promoted to fp64; x = a*H + b with a*H and +b rounded separately.
+   Bhat = ceil(min(N, max(Bmin, e^x))) with e^x evaluated in 113-bit binary128
+   (libquadmath), so the ceiling is the exact one: for a double x != 0, e^x
+   is irrational and lies farther than 2^-113 relative from every integer in
+   practice, while an fp64 exponential can land on the wrong side of an
+   integer it is within a few ulps of (e.g. a = 0, b = ln k).  One case is
+   below binary128's resolution: for 0 < x < 2^-113, e^x = 1 + x + ... rounds
+   to 1, while e^x > 1 for every x > 0, so its ceiling is 2.  x = NaN gives
+   Bmin. */
 int64_t oracle_budget(float Hent, double a, double b, int64_t N, int64_t Bmin)
 {
     volatile double ah = a * (double)Hent;
     volatile double x = ah + b;
-    double e = exp(x);
-    double B = fmin((double)N, fmax((double)Bmin, e));
-    return (int64_t)ceil(B);
+    if (isnan(x)) return Bmin;
+    __float128 c = ceilq(expq((__float128)x));
+    if (x > 0 && c < 2) c = 2;
+    if (c < (__float128)Bmin) c = (__float128)Bmin;
+    if (c > (__float128)N) c = (__float128)N;
+    return (int64_t)c;
 }
 
 /* E3 + E4 per (head, token).  Hent[row] is the fp32 entropy of query

@@ -9,9 +9,14 @@
 // softmax attention under the radius mask.
 //
 // One CTA per pair of query tiles (A = tile 2p, B = tile 2p+1) of one head.
-// The two tiles' key-tile lists are merged (a sorted union with per-tile
-// "listed" and "full" flags); each merged key tile is loaded once and used by
-// whichever of A and B lists it.  384 threads:
+// The two tiles' key-tile lists are merged (a union with per-tile "listed" and
+// "full" flags); each merged key tile is loaded once and used by whichever of
+// A and B lists it.  The merged order puts the tiles only one of A and B
+// lists first, alternating A-only and B-only, then the tiles both list: the
+// two query tiles then work on different key tiles at the same time instead
+// of one idling while the other's own tiles stream past (the two rings are
+// only two tiles deep), so a CTA takes about max(|A|, |B|) chain steps rather
+// than |A u B|.  384 threads:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
 //              warpgroup owns query row r (TMEM lane r).  Reads S from TMEM,
 //              applies the token mask as an additive 0 / -inf bias (per key
@@ -22,15 +27,17 @@
 //              fp32x2 arithmetic.
 //              The two warpgroups work on independent tiles, so one computes
 //              while the other waits for the tensor core.
-//   warp 8     TMA producer: Q_A, Q_B, then the K and V rings.
+//   warp 8     TMA producer: Q_A, Q_B, then the K ring.
+//   warp 11    TMA producer of the V ring (its own thread, so K tiles run
+//              ahead as far as the K ring allows, whatever the V ring waits on).
 //   warps 9,10 MMA issuers for tiles A and B (warp 9 also allocates TMEM): for
 //              each listed key tile j, O_w += P_w(j) V(j), and in the same issue
 //              group S_w = Q_w K(j')^T for the next listed tile j' once its K
 //              has landed (the tensor pipe runs one thread's MMAs in order, so
 //              the QK overwrites S, where P_w lives, only after the PV has read
 //              it); the two tiles progress independently.
-//   warp 11    idle (completes the third warpgroup for register rebalancing:
-//              the softmax warpgroups run with 216 registers, warps 8-11 with 72).
+//   Register rebalancing: the softmax warpgroups run with 216 registers,
+//   warps 8-11 with 72.
 // With radius-sorted query groups the CTA takes two mask slots instead (slot s
 // of frames 2f and 2f+1), stages the Q tiles of both pairs in the idle K/V
 // rings and copies each slot's 128 query rows into slot order before the
@@ -55,7 +62,8 @@ struct AttnCfg {
     static constexpr int OFF_V = OFF_K + KST * TILE;
     static constexpr int OFF_DYN = OFF_V + VST * TILE;      // lists, half-widths, bitmaps, barriers
     static constexpr int WARP_LOAD = 8, WARP_MMA = 9;       // MMA issuers: warps 9 (tile A), 10 (tile B)
-    static constexpr int THREADS = 384;                     // warp 11 only completes warpgroup 2
+    static constexpr int WARP_VLOAD = 11;                   // V-ring producer
+    static constexpr int THREADS = 384;
     // registers after rebalancing: softmax warpgroups 0, 1 and warpgroup 2
     // (384 x 168 at launch = 2 x 128 x 216 + 128 x 72)
     static constexpr int REGS_SOFTMAX = 216, REGS_OTHER = 72;
@@ -75,10 +83,10 @@ struct AttnDyn {
         L.bw = ((2 * rte + 2) * tiles_per_frame + 31) / 32;
         L.merged = 0;                                               // uint32 [2 * list_cap]
         L.stab = L.merged + 8 * list_cap;                           // uint16 [2][rte + 1][128]
-        L.bits = L.stab + ((2 * (rte + 1) * 128 * 2 + 15) & ~15);   // uint32 [5][bw]
-        L.bars = L.bits + ((5 * L.bw * 4 + 15) & ~15);              // uint64 [32]
+        L.bits = L.stab + ((2 * (rte + 1) * 128 * 2 + 15) & ~15);   // uint32 [7][bw]
+        L.bars = L.bits + ((7 * L.bw * 4 + 15) & ~15);              // uint64 [32]
         L.misc = L.bars + 8 * 32;
-        L.total = L.misc + 16;
+        L.total = L.misc + 32;
         return L;
     }
 };
@@ -111,7 +119,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t* dyn = smem + C::OFF_DYN;
     uint32_t* merged = reinterpret_cast<uint32_t*>(dyn + L.merged);
     uint16_t* s_tab = reinterpret_cast<uint16_t*>(dyn + L.stab);
-    uint32_t* bits = reinterpret_cast<uint32_t*>(dyn + L.bits);      // [5][bw]
+    // [7][bw]: listed by A, by B, full for A, full for B, then the word
+    // offsets of the A-only, B-only and both-listed classes
+    uint32_t* bits = reinterpret_cast<uint32_t*>(dyn + L.bits);
     uint64_t* bars = reinterpret_cast<uint64_t*>(dyn + L.bars);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
@@ -126,6 +136,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     volatile int* s_abort = reinterpret_cast<volatile int*>(dyn + L.misc + 4);
     int* s_n = reinterpret_cast<int*>(dyn + L.misc + 8);
     int* s_lock = reinterpret_cast<int*>(dyn + L.misc + 12);
+    int* s_cls = reinterpret_cast<int*>(dyn + L.misc + 16);         // [2]: A-only and B-only counts
 
     const int pair = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,18 +158,21 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         nA = 0;
         nB = 0;
     }
-    const int ta = qa / G.tiles_per_frame;
+    const int ta = qa / G.tiles_per_frame, tb = qb / G.tiles_per_frame;
     const int base = max(0, ta - G.rte) * G.tiles_per_frame;   // first key tile either list can hold
 
-    // ---- merge the two sorted lists: set bits, scan word counts, expand in order
-    for (int i = tid; i < 5 * L.bw; i += C::THREADS) bits[i] = 0;
+    // ---- merge the two sorted lists: set bits, scan per-class word counts,
+    // expand (A-only and B-only alternating, then the tiles both list)
+    for (int i = tid; i < 7 * L.bw; i += C::THREADS) bits[i] = 0;
     __syncthreads();
     for (int i = tid; i < nA + nB; i += C::THREADS) {
         const bool isB = i >= nA;
         const int e = isB ? lists[(size_t)qb * G.list_cap + (i - nA)] : lists[(size_t)qa * G.list_cap + i];
         const int bit = (e & 0x7fff) - base;
-        // a key tile no query of the pair can reach is an error: recorded, skipped
-        if (bit < 0 || bit >= 32 * L.bw || (e & 0x7fff) >= G.nQ) {
+        // a key tile its own query tile cannot reach (outside the grid, or more
+        // than Rt' frames from that tile's frame) is an error: recorded, skipped
+        const int fe = (e & 0x7fff) / G.tiles_per_frame;
+        if (bit < 0 || bit >= 32 * L.bw || (e & 0x7fff) >= G.nQ || abs(fe - (isB ? tb : ta)) > G.rte) {
             atomicOr(&g_tra_error, TRA_ERRBIT_CHECK);
             continue;
         }
@@ -167,33 +181,53 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     __syncthreads();
     if (warp == 0) {
-        int carry = 0;
+        int carry[3] = {0, 0, 0};
         for (int w0 = 0; w0 < L.bw; w0 += 32) {
             const int w = w0 + lane;
-            const int c = w < L.bw ? __popc(bits[w] | bits[L.bw + w]) : 0;
-            int incl = c;
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
+            const uint32_t ia = w < L.bw ? bits[w] : 0u, ib = w < L.bw ? bits[L.bw + w] : 0u;
+            const uint32_t cls[3] = {ia & ~ib, ib & ~ia, ia & ib};
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                const int cnt = __popc(cls[c]);
+                int incl = cnt;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                if (w < L.bw) bits[(4 + c) * L.bw + w] = carry[c] + incl - cnt;
+                carry[c] += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (w < L.bw) bits[4 * L.bw + w] = carry + incl - c;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) *s_n = carry;
+        if (lane == 0) {
+            s_cls[0] = carry[0];
+            s_cls[1] = carry[1];
+            *s_n = carry[0] + carry[1] + carry[2];
+        }
     }
     __syncthreads();
-    for (int w = tid; w < L.bw; w += C::THREADS) {
-        const uint32_t ia = bits[w], ib = bits[L.bw + w], fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
-        uint32_t m = ia | ib;
-        int pos = (int)bits[4 * L.bw + w];
-        while (m) {
-            const int b = __ffs(m) - 1;
-            m &= m - 1;
-            int tk, trk, tck;
-            tile_coords(G, base + 32 * w + b, tk, trk, tck);
-            const uint32_t bit = 1u << b;
-            merged[pos++] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) | ((ib & bit) ? (MT_IN0 << 1) : 0u) |
-                            ((fa & bit) ? MT_FULL0 : 0u) | ((fb & bit) ? (MT_FULL0 << 1) : 0u);
+    {
+        const int nAo = s_cls[0], nBo = s_cls[1], m2 = min(nAo, nBo);
+        for (int w = tid; w < L.bw; w += C::THREADS) {
+            const uint32_t ia = bits[w], ib = bits[L.bw + w], fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                uint32_t m = c == 0 ? (ia & ~ib) : (c == 1 ? (ib & ~ia) : (ia & ib));
+                int k = (int)bits[(4 + c) * L.bw + w];      // rank of the word's first entry in its class
+                while (m) {
+                    const int b = __ffs(m) - 1;
+                    m &= m - 1;
+                    // A-only rank k goes to 2k, B-only to 2k + 1 while both
+                    // classes last; the longer one's rest follows; then both
+                    const int pos = c == 2 ? nAo + nBo + k : (k < m2 ? 2 * k + c : m2 + k);
+                    ++k;
+                    int tk, trk, tck;
+                    tile_coords(G, base + 32 * w + b, tk, trk, tck);
+                    const uint32_t bit = 1u << b;
+                    merged[pos] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) |
+                                  ((ib & bit) ? (MT_IN0 << 1) : 0u) | ((fa & bit) ? MT_FULL0 : 0u) |
+                                  ((fb & bit) ? (MT_FULL0 << 1) : 0u);
+                }
+            }
         }
     }
     if (tid == 0) {
@@ -255,11 +289,17 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (warp >= C::WARP_LOAD) {
       regs_dec<C::REGS_OTHER>();
-      if (warp == C::WARP_LOAD) {
-        // ------------------------------------------------ TMA producer: Q_A, Q_B, K and V rings
+      if (warp == C::WARP_LOAD || warp == C::WARP_VLOAD) {
+        // ------------------------------------------------ TMA producers: Q_A, Q_B and the K ring
+        // (warp 8), the V ring (warp 11); each walks the merged list on its own
+        const bool isK = warp == C::WARP_LOAD;
         if (lane == 0 && n > 0) {
-            prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
-            if (!G.qsort) {                                         // else staged and gathered above
+            if (isK) {
+                prefetch_tmap(&tm_q); prefetch_tmap(&tm_k);
+            } else {
+                prefetch_tmap(&tm_v);
+            }
+            if (isK && !G.qsort) {                                  // else staged and gathered above
                 mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
                 int tqa, trqa, tcqa, tqb, trqb, tcqb;
                 tile_coords(G, qa, tqa, trqa, tcqa);
@@ -270,28 +310,27 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (hasB) load_tile_panel(sQ + C::TILE + p * C::PANEL, &tm_q, G, p, g, tqb, trqb, tcqb, q_full);
                 }
             }
-            int kiss = 0, viss = 0;
+            static_assert(C::KST == C::VST, "one ring depth for K and V");
+            constexpr int ST = C::KST;
+            uint64_t* fullb = isK ? k_full : v_full;
+            uint64_t* emptyb = isK ? k_empty : v_empty;
+            uint8_t* ring = isK ? sK : sV;
+            const CUtensorMap* tm = isK ? &tm_k : &tm_v;
+            int iss = 0;
             for (int j = 0; j < n; ++j) {
                 const uint32_t e = merged[j];
                 const int tk = (int)(e & 0x7fff), trk = (int)((e >> 15) & 63), tck = (int)((e >> 21) & 31);
-                const int ks = j % C::KST, vs = j % C::VST;
-                if (j >= C::KST && !role_wait(&k_empty[ks], ((j / C::KST) - 1) & 1, G.wait_ns, s_abort)) break;
-                mbar_arrive_expect_tx(&k_full[ks], C::TILE);
+                const int st = j % ST;
+                if (j >= ST && !role_wait(&emptyb[st], ((j / ST) - 1) & 1, G.wait_ns, s_abort)) break;
+                mbar_arrive_expect_tx(&fullb[st], C::TILE);
 #pragma unroll
                 for (int p = 0; p < C::NP; ++p)
-                    load_tile_panel(sK + ks * C::TILE + p * C::PANEL, &tm_k, G, p, g, tk, trk, tck, &k_full[ks]);
-                ++kiss;
-                if (j >= C::VST && !role_wait(&v_empty[vs], ((j / C::VST) - 1) & 1, G.wait_ns, s_abort)) break;
-                mbar_arrive_expect_tx(&v_full[vs], C::TILE);
-#pragma unroll
-                for (int p = 0; p < C::NP; ++p)
-                    load_tile_panel(sV + vs * C::TILE + p * C::PANEL, &tm_v, G, p, g, tk, trk, tck, &v_full[vs]);
-                ++viss;
+                    load_tile_panel(ring + st * C::TILE + p * C::PANEL, tm, G, p, g, tk, trk, tck, &fullb[st]);
+                ++iss;
             }
             // copies still in flight must land before the CTA exits
-            mbar_wait(q_full, 0, G.drain_ns);
-            for (int j = max(0, kiss - C::KST); j < kiss; ++j) mbar_wait(&k_full[j % C::KST], (j / C::KST) & 1, G.drain_ns);
-            for (int j = max(0, viss - C::VST); j < viss; ++j) mbar_wait(&v_full[j % C::VST], (j / C::VST) & 1, G.drain_ns);
+            if (isK) mbar_wait(q_full, 0, G.drain_ns);
+            for (int j = max(0, iss - ST); j < iss; ++j) mbar_wait(&fullb[j % ST], (j / ST) & 1, G.drain_ns);
         }
       } else if (warp == C::WARP_MMA || warp == C::WARP_MMA + 1) {
         // ------------------------------------------------ MMA issuers, one per query tile
@@ -324,14 +363,28 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mma_commit(&s_full[w]);
                 mma_commit(&k_empty[kss]);
             };
+            // An entry this tile does not list is released as soon as its K has
+            // landed; its V stage is released one step later (at the next entry,
+            // after that entry's QK has gone out), so a V tile that lands late
+            // never holds up this tile's next QK.  At most one V release is
+            // pending, so the V ring always moves on.
+            int pend_v = -1;
+            auto release_v = [&]() -> bool {
+                if (pend_v < 0) return true;
+                const int pj = pend_v;
+                pend_v = -1;
+                if (!role_wait(&v_full[pj % C::VST], (pj / C::VST) & 1, G.wait_ns, s_abort)) return false;
+                mbar_arrive(&v_empty[pj % C::VST]);
+                return true;
+            };
             for (int j = 0; ok && j < n; ++j) {
                 const bool uses = (merged[j] & in_bit) != 0;
                 const int ks = j % C::KST, vs = j % C::VST;
                 if (!uses) {
+                    if (!release_v()) { ok = false; break; }
                     if (!role_wait(&k_full[ks], (j / C::KST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                     mbar_arrive(&k_empty[ks]);
-                    if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
-                    mbar_arrive(&v_empty[vs]);
+                    pend_v = j;
                     continue;
                 }
                 if (qk_ahead != j) {
@@ -341,6 +394,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     issue_qk(j);
                     issue_unlock(s_lock);
                 }
+                if (!release_v()) { ok = false; break; }
                 if (!role_wait(&p_full[w], cnt & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
@@ -352,19 +406,23 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                            (cnt > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&pv_done[w]);
                 mma_commit(&v_empty[vs]);
-                // The next tile's QK joins this group when this query tile lists
-                // it and its K has landed: the tensor pipe runs the MMAs of one
-                // thread in order, so the QK overwrites S (holding P) only after
-                // this PV has read P.
-                if (j + 1 < n && (merged[j + 1] & in_bit) &&
-                    mbar_test(&k_full[(j + 1) % C::KST], ((j + 1) / C::KST) & 1)) {
+                // This tile's next listed entry j' joins this group when its K has
+                // landed: the tensor pipe runs the MMAs of one thread in order, so
+                // the QK overwrites S (holding P) only after this PV has read it.
+                // Only j' <= j + KST is looked at: every earlier entry of j''s
+                // ring stage has then been waited for by this thread, so the
+                // parity test names j''s own landing.
+                int jn = j + 1;
+                while (jn < n && jn <= j + C::KST && !(merged[jn] & in_bit)) ++jn;
+                if (jn < n && jn <= j + C::KST && mbar_test(&k_full[jn % C::KST], (jn / C::KST) & 1)) {
                     tc_fence_after();
-                    issue_qk(j + 1);
-                    qk_ahead = j + 1;
+                    issue_qk(jn);
+                    qk_ahead = jn;
                 }
                 issue_unlock(s_lock);
                 ++cnt;
             }
+            if (ok && !release_v()) ok = false;
             // every issued MMA must finish before TMEM is freed
             mma_commit(&drain[w]);
             mbar_wait(&drain[w], 0, G.drain_ns);

@@ -42,13 +42,6 @@ struct EntCfg {
     static constexpr int WARP_LOAD = 8, WARP_MMA = 9;     // MMA issuers: warps 9 (tile A), 10 (tile B)
 };
 
-// With ENT_POLY_MOD = p > 0, exp2 of the element pairs with pair % p == p - 1
-// runs on the FMA pipe (degree-4 polynomial, packed pairs) and the rest on the
-// MUFU unit.  Measured at Wan-720p shapes (dense, 40 heads): p = 0 (every
-// exponential on MUFU) 85.4 ms, p = 6 85.5, p = 4 88.6, p = 3 92.9, p = 2
-// 101.6; the FMA pipe is the busier one, so the split is off.
-constexpr int ENT_POLY_MOD = 0;
-
 // One key tile's contribution to a query row's online entropy statistics in
 // the log2 domain: m = running maximum of s*c, Z = sum 2^(s*c - m), A = sum
 // 2^(s*c - m) * (s*c - m); the entropy is then ln Z - ln2 * A / Z.  v holds the
@@ -84,15 +77,9 @@ __device__ __forceinline__ void ent_tile_update(uint32_t (&v)[4][32], bool edge,
     for (int i = 0; i < 64; ++i) {
         const f2_t u2 = f2_fma(f2_pack(__uint_as_float(v[i >> 4][(2 * i) & 31]),
                                        __uint_as_float(v[i >> 4][(2 * i + 1) & 31])), c2, nm2);
-        f2_t e2;
-        constexpr int PD = ENT_POLY_MOD > 0 ? ENT_POLY_MOD : 1;
-        if (ENT_POLY_MOD > 0 && i % PD == PD - 1) {
-            e2 = ex2_poly4_pair(u2);
-        } else {
-            float u0, u1;
-            f2_unpack(u2, u0, u1);
-            e2 = f2_pack(ex2(u0), ex2(u1));
-        }
+        float u0, u1;
+        f2_unpack(u2, u0, u1);
+        const f2_t e2 = f2_pack(ex2(u0), ex2(u1));
         z2[i & 3] = f2_add(z2[i & 3], e2);
         a2[i & 3] = f2_fma(e2, u2, a2[i & 3]);
     }

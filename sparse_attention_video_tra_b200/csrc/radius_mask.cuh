@@ -10,7 +10,8 @@
 // never changes the attention output.
 //
 // One CTA per (query tile, head), one thread per tile row (token).
-//   1. Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))) in fp64.
+//   1. Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))), y = a*H + b in fp64 and
+//      the ceiling of e^y decided exactly.
 //   2. r = the smallest r in [0, r_cap] whose clipped neighbourhood count
 //      reaches Bhat (binary search; the count is monotone in r).
 //   3. Per frame distance |dt|: every query's neighbourhood is a rectangle of
@@ -27,6 +28,7 @@
 // step 3 still holds because every member's rectangle contains its own tile
 // column, one of two adjacent columns of the same tile row.
 #pragma once
+#include "exact_budget.cuh"
 #include "tra_common.cuh"
 
 namespace tra {
@@ -64,12 +66,12 @@ __device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int 
     return c;
 }
 
+// Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))): a*H and + b rounded
+// separately in fp64, the ceiling decided exactly (exact_budget.cuh)
 __device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
 {
-    const double x = __dadd_rn(__dmul_rn(G.a, (double)Hent), G.b);
-    const double e = exp(x);
-    const double B = fmin((double)G.N, fmax((double)G.Bmin, e));
-    return (long long)ceil(B);
+    const double y = __dadd_rn(__dmul_rn(G.a, (double)Hent), G.b);
+    return budget_from_exponent(y, G.N, G.Bmin);
 }
 
 // r = the smallest r in [0, r_cap] whose neighbourhood count reaches bh (the

@@ -254,29 +254,6 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// 2^x on the FMA pipe, for x <= 127 (x <= -127 gives exactly 0): round x to
-// an integer k by adding 1.5*2^23 (+127, the exponent bias) so that k sits in
-// the low mantissa bits, take f = x - k in [-1/2, 1/2], evaluate a polynomial
-// fitted to 2^f on that interval (minimax in relative error, coefficients
-// computed for this library), and scale by 2^k built from the same bits.
-// Relative error: 7.5e-5 (degree 3), 2.7e-6 (degree 4).
-template <int DEG>
-__device__ __forceinline__ float ex2_poly(float x)
-{
-    x = fmaxf(x, -127.0f);
-    const float t = x + 12583039.0f;                 // 1.5 * 2^23 + 127
-    const float f = x - (t - 12583039.0f);           // x - round(x)
-    float p;
-    if constexpr (DEG == 3) {
-        p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-    } else {
-        p = fmaf(fmaf(fmaf(fmaf(0.0095701013f, f, 0.0559178591f), f, 0.2402474433f), f, 0.6931217909f), f,
-                 0.9999992847f);
-    }
-    const float scale = __int_as_float(__float_as_int(t) << 23);   // 2^k, 0 when k = -127
-    return p * scale;
-}
-
 // ---- packed fp32 pairs (sm_100 FFMA2/FADD2/FMUL2): two floats in a 64-bit register
 typedef unsigned long long f2_t;
 
@@ -311,26 +288,6 @@ __device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b)
     f2_t r;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
-}
-
-// 2^x for a pair, on the FMA pipe (the same method as ex2_poly<4>), for
-// x <= 0 (x <= -127 gives exactly 0).
-__device__ __forceinline__ f2_t ex2_poly4_pair(f2_t x2)
-{
-    float a, b;
-    f2_unpack(x2, a, b);
-    x2 = f2_pack(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
-    const f2_t C = f2_pack(12583039.0f, 12583039.0f);        // 1.5 * 2^23 + 127
-    const f2_t t = f2_add(x2, C);                                // round(x) in the low mantissa bits
-    const f2_t f = f2_add(x2, f2_fma(t, f2_pack(-1.0f, -1.0f), C));   // x - round(x), exact
-    f2_t p = f2_fma(f2_pack(0.0095701013f, 0.0095701013f), f, f2_pack(0.0559178591f, 0.0559178591f));
-    p = f2_fma(p, f, f2_pack(0.2402474433f, 0.2402474433f));
-    p = f2_fma(p, f, f2_pack(0.6931217909f, 0.6931217909f));
-    p = f2_fma(p, f, f2_pack(0.9999992847f, 0.9999992847f));
-    float t0, t1;
-    f2_unpack(t, t0, t1);
-    const f2_t scale = f2_pack(__int_as_float(__float_as_int(t0) << 23), __int_as_float(__float_as_int(t1) << 23));
-    return f2_mul(p, scale);
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c)

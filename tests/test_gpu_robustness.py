@@ -71,6 +71,27 @@ def test_unreachable_list_entry_is_reported_and_skipped():
     assert plan.status() == 6
 
 
+def test_list_entry_beyond_its_own_tiles_reach_is_reported():
+    """A listed key tile Rt' + 1 frames from the query tile that lists it is
+    still inside the range of key tiles the CTA's pair of query tiles could
+    reach together, so it must be caught by the per-list frame check (the
+    half-width table has no row for that frame distance)."""
+    plan, (qt, kt, vt), _, mask = _setup()
+    i = plan.info
+    tpf = i.n_tiles_h * i.n_tiles_w
+    assert i.rt_eff + 1 < i.T
+    bad = mask.clone()
+    lst = plan.mask_views(bad)[3]
+    lst[0, 0, 0] = (i.rt_eff + 1) * tpf              # frame Rt'+1; tile 0 sits in frame 0
+    out = plan.new_out()
+    plan.attention(qt, kt, vt, bad, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 6
+    plan.attention(qt, kt, vt, mask, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+
+
 def test_results_are_bit_identical_across_runs():
     plan, (qt, kt, vt), Ht, mask = _setup(seed=9)
     i = plan.info

@@ -27,7 +27,8 @@ MUTANTS = [
      1, [f"{PINS}::test_rt_eff_and_r_cap"]),
     ("temporal reach one frame short", "for (int dt = -rte; dt <= rte; ++dt) {", "for (int dt = -rte; dt < rte; ++dt) {",
      1, [f"{PINS}::test_count_equals_bruteforce_mask_rows"]),
-    ("budget floored instead of ceiled", "    return (int64_t)ceil(B);\n}", "    return (int64_t)floor(B);\n}", 1,
+    ("budget floored instead of ceiled", "__float128 c = ceilq(expq((__float128)x));",
+     "__float128 c = floorq(expq((__float128)x));", 1,
      [f"{PINS}::test_budget_closed_forms"]),
     ("radius scan stops one early", "while (c < bh && r < rcap) {", "while (c < bh - 1 && r < rcap) {", 1,
      [f"{PINS}::test_radius_matches_bruteforce"]),
@@ -51,6 +52,9 @@ MUTANTS = [
       "tests/test_oracle_qsort_pins.py::test_sets_equal_bruteforce"]),
     ("calibration cut one key late", "if (cum >= mass) { kk = j + 1; break; }", "if (cum > mass) { kk = j + 2; break; }", 1,
      [f"{CALIB}::test_uniform_attention_needs_ceil_mass_times_n", f"{CALIB}::test_topk_matches_numpy_sort"]),
+    ("budget ceiling from an fp64 exponential", "__float128 c = ceilq(expq((__float128)x));",
+     "__float128 c = ceilq((__float128)exp(x));", 1,
+     ["tests/test_budget_exact.py::test_oracle_budget_is_the_exact_ceiling_near_integers"]),
     ("calibration fit through the origin (no intercept)", "double dx = H[i] - mx, dy = fit_y(k[i]) - my;",
      "double dx = H[i], dy = fit_y(k[i]);", 1,
      [f"{CALIB}::test_fit_hand_worked_three_points", f"{CALIB}::test_fit_matches_numpy_polyfit_on_noisy_data"]),
