@@ -426,19 +426,22 @@ def _oracle_calibrate_b(oracle, wl, dev):
 
 
 def query_group_flags(mode: str, wl) -> int:
-    """TRA_FLAG_QSORT when asked for, or (auto) when the workload's frame has
-    an even number of tile columns, so that a pair of query tiles is two
-    side-by-side tiles (the plan refuses the flag otherwise)."""
+    """TRA_FLAG_QSORT when asked for, or (auto) when the plan accepts it and a
+    frame has more than one tile row, so that a tile-column strip holds
+    several tiles whose queries can be regrouped by radius (with one tile row
+    the groups are the tiles themselves)."""
     from sparse_attention_video_tra_b200 import Plan, TRA_FLAG_QSORT, TraError
     if mode == "off":
         return 0
     try:
-        Plan(wl.T, wl.H, wl.W, 1, wl.d, wl.a, 0.0, wl.gamma, wl.Rt, wl.Bmin, TRA_FLAG_QSORT).close()
+        p = Plan(wl.T, wl.H, wl.W, 1, wl.d, wl.a, 0.0, wl.gamma, wl.Rt, wl.Bmin, TRA_FLAG_QSORT)
+        rows = p.info.n_tiles_h
+        p.close()
     except TraError:
         if mode == "on":
             raise
         return 0
-    return TRA_FLAG_QSORT
+    return TRA_FLAG_QSORT if (mode == "on" or rows > 1) else 0
 
 
 def run_tra(args, rank, world):

@@ -105,16 +105,18 @@ typedef enum {
                                               s(r, Rt')^2 >= (H-1)^2 + (W-1)^2. */
 #define TRA_FLAG_QSORT         (1u << 20)  /* radius-sorted query groups (a scheduling
                                               choice of this library; the results are
-                                              the same attention): the 256 queries of
-                                              each pair of query tiles (2p, 2p+1) are
-                                              ordered by (radius, tile-major row), pad
-                                              rows first, and the first 128 take the
-                                              block-mask slot of tile 2p, the rest that
-                                              of tile 2p+1.  Each group's key-tile list
-                                              is the union over its own queries, so
-                                              fewer tile pairs are computed.  Needs an
-                                              even number of tile columns per frame
-                                              (a pair is then two side-by-side tiles);
+                                              the same attention): the rows of each
+                                              tile-column strip (one tile column of
+                                              one frame: its n_tiles_h tiles, top to
+                                              bottom, strip row l = 128*u + i for row
+                                              i of the tile in tile row u) are ordered
+                                              by (radius, l), pad rows first, and the
+                                              u-th block of 128 takes the block-mask
+                                              slot of the strip's tile in tile row u.
+                                              Each group's key-tile list is the union
+                                              over its own queries, so a group of like
+                                              radii computes fewer tile pairs than a
+                                              spatial tile.  Needs n_tiles_h <= 4;
                                               otherwise TRA_ERR_UNSUPPORTED. */
 
 /* everything a caller needs to size and read buffers */
@@ -135,11 +137,11 @@ typedef struct {
        tile_pairs int64  [heads][n_tiles]      sum of c_i(r_i) over the tile's queries
        list       uint16 [heads][n_tiles][list_cap]  active key-tile indices in
                   ascending order; bit 15 set = full tile (no token inside is masked)
-       group      uint8  [heads][n_tiles][128]  TRA_FLAG_QSORT only: the query of
-                  each slot of the tile's group as a row 0..255 of its pair
-                  (rows 0..127 = tile 2p, 128..255 = tile 2p+1); tile_count,
-                  tile_pairs and list then describe the group, not the tile.
-                  off_group = 0 without the flag. */
+       group      uint16 [heads][n_tiles][128]  TRA_FLAG_QSORT only: the query of
+                  each slot of the tile's group as a strip row l (row l % 128
+                  of the tile in tile row l / 128 of the same tile column and
+                  frame); tile_count, tile_pairs and list then describe the
+                  group, not the tile.  off_group = 0 without the flag. */
     size_t off_radius, off_tile_count, off_tile_pairs, off_list;
     size_t off_group;
 } tra_plan_info;

@@ -191,40 +191,43 @@ def block_mask(r, G, grid, gamma, Rt, qtile, ktile, qtiles=None, metric: int = C
 def query_groups(r, G, grid, tile):
     """The radius-sorted query groups of TRA_FLAG_QSORT plans (a design of this
     library, not of the pages).  Query tiles are (1, th, tw) boxes in the
-    tile-major order; tiles 2p and 2p+1 of a head form a pair.  The pair's
-    256 tile-major rows are ordered by (radius, row) with pad rows (outside the
-    grid, radius -1) first; the first 128 are the group of tile 2p, the rest
-    that of tile 2p+1.
+    tile-major order.  A strip is one tile column of one frame: its nTh tiles,
+    top to bottom, hold strip rows l = u*128 + i (row i of the tile in tile
+    row u).  The strip's rows are ordered by (radius, l), pad rows (outside the
+    grid, radius -1) first, and the u-th block of 128 is the group that takes
+    the mask slot of the strip's tile in tile row u.
 
     r: int32 radii [G*N] in natural order.  Returns
-      perm    uint8 [G, nQ, 128]: pair-local row (0..255) of each group slot;
+      perm    uint16 [G, nQ, 128]: strip row (0 .. 128*nTh - 1) of each group slot;
       members int64 [G*nQ, 128]: the slot's query as g*N + n, -1 on pad rows."""
     T, H, W = grid
     th, tw = tile
     nTh, nTw = -(-H // th), -(-W // tw)
-    nQ = T * nTh * nTw
-    assert nQ % 2 == 0, "pairs need an even number of query tiles"
+    tpf = nTh * nTw
+    nQ = T * tpf
     N = T * H * W
     rr = np.asarray(r, dtype=np.int64).reshape(G, N)
     p = np.arange(nQ * 128)
     tile, inn = p // 128, p % 128
-    t, rem = tile // (nTh * nTw), tile % (nTh * nTw)
+    t, rem = tile // tpf, tile % tpf
     h = (rem // nTw) * th + inn // tw
     w = (rem % nTw) * tw + inn % tw
     valid = (h < H) & (w < W)
     nat = np.where(valid, (t * H + h) * W + w, -1)
-    perm = np.zeros((G, nQ, 128), np.uint8)
+    perm = np.zeros((G, nQ, 128), np.uint16)
     members = np.full((G * nQ, 128), -1, np.int64)
     for g in range(G):
         rad = np.where(valid, rr[g][np.maximum(nat, 0)], -1)
-        for a in range(0, nQ, 2):
-            rows = np.arange(a * 128, a * 128 + 256)
-            order = np.argsort(rad[rows], kind="stable")        # (radius, row): stable on row
-            for k in range(2):
-                sl = order[128 * k:128 * (k + 1)]
-                perm[g, a + k] = sl
-                src = nat[rows[sl]]
-                members[g * nQ + a + k] = np.where(src >= 0, g * N + src, -1)
+        for tt in range(T):
+            for c in range(nTw):
+                tiles = [tt * tpf + u * nTw + c for u in range(nTh)]
+                rows = np.concatenate([np.arange(a * 128, a * 128 + 128) for a in tiles])   # strip row l -> tile-major row
+                order = np.argsort(rad[rows], kind="stable")        # (radius, l): stable on l
+                for u, a in enumerate(tiles):
+                    sl = order[128 * u:128 * (u + 1)]
+                    perm[g, a] = sl
+                    src = nat[rows[sl]]
+                    members[g * nQ + a] = np.where(src >= 0, g * N + src, -1)
     return perm, members
 
 

@@ -267,14 +267,14 @@ class Plan:
         return bool(self.flags & TRA_FLAG_QSORT)
 
     def group_view(self, mask):
-        """TRA_FLAG_QSORT: uint8 [heads, n_tiles, 128], the pair row (0..255)
-        of each slot of each tile's query group."""
+        """TRA_FLAG_QSORT: [heads, n_tiles, 128] int16 view of the uint16 strip
+        row (0 .. 128*n_tiles_h - 1) of each slot of each tile's query group."""
         import torch
         i = self.info
         if not self.qsort:
             raise ValueError("the plan has no query groups (TRA_FLAG_QSORT)")
-        n = i.heads * i.n_tiles * 128
-        return mask[i.off_group:i.off_group + n].view(torch.uint8).view(i.heads, i.n_tiles, 128)
+        n = i.heads * i.n_tiles * 128 * 2
+        return mask[i.off_group:i.off_group + n].view(torch.int16).view(i.heads, i.n_tiles, 128)
 
     def mask_views(self, mask):
         """(radius [heads,N_pad] i32, tile_count [heads,n_tiles] i32,

@@ -39,10 +39,10 @@
 //   Register rebalancing: the softmax warpgroups run with 216 registers,
 //   warps 8-11 with 72.
 // With radius-sorted query groups the CTA takes two mask slots instead (slot s
-// of frames 2f and 2f+1), stages the Q tiles of both pairs in the idle K/V
-// rings and copies each slot's 128 query rows into slot order before the
-// roles start; each softmax thread then speaks for its slot's query and
-// writes that query's output row.
+// of frames 2f and 2f+1: groups of like radius), gathers each slot's 128 query
+// rows (rows of its tile-column strip) from global memory straight into the Q
+// tiles before the roles start; each softmax thread then speaks for its slot's
+// query and writes that query's output row.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512)
 // (P_A, P_B as bf16 pairs in the first 64 columns of S_A, S_B).
 #pragma once
@@ -109,7 +109,7 @@ template <int D, int TWL, bool OUT_BF16, bool DISK>
 __global__ void __launch_bounds__(384, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const Geom G, const uint8_t* __restrict__ mask,
-                 void* __restrict__ out)
+                 void* __restrict__ out, const void* __restrict__ qraw)
 {
     using C = AttnCfg<D>;
     constexpr int TW = 1 << TWL;
@@ -250,38 +250,33 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t* sK = smem + C::OFF_K;
     uint8_t* sV = smem + C::OFF_V;
     const int kbase = g * G.N_pad;
-    // radius-sorted query groups: row r of slot s holds pair row grp_s[r] of
-    // the pair (tiles s & ~1 and (s & ~1) + 1)
-    const uint8_t* grp_a = mask + G.off_group + ((size_t)g * G.nQ + qa) * 128;
-    const uint8_t* grp_b = grp_a + (size_t)(qb - qa) * 128;
+    // radius-sorted query groups: row r of slot s holds strip row grp_s[r] of
+    // the slot's strip (tile row grp >> 7, row grp & 127 of that tile)
+    const uint16_t* grp_a = reinterpret_cast<const uint16_t*>(mask + G.off_group) + ((size_t)g * G.nQ + qa) * 128;
+    const uint16_t* grp_b = grp_a + (size_t)(qb - qa) * 128;
     if (G.qsort && n > 0) {
-        // Q of both pairs lands in the idle K and V rings (four tiles, one
-        // pair without slot B), then each slot's rows are copied into
-        // slot order (128-byte swizzle on both sides)
-        static_assert(C::OFF_V == C::OFF_K + C::KST * C::TILE && C::KST + C::VST >= 4, "staging space");
+        // gather both slots' query rows into Q_A / Q_B (128-byte swizzle),
+        // 16 bytes per load; rows outside the grid are zeros
+        constexpr int CH = D / 8;                           // 16-byte chunks of a row
         const int np = hasB ? 2 : 1;
-        if (warp == C::WARP_LOAD && lane == 0) {
-            prefetch_tmap(&tm_q);
-            mbar_arrive_expect_tx(q_full, 2 * np * C::TILE);
-            for (int k = 0; k < 2 * np; ++k) {
-                int tq, trq, tcq;
-                tile_coords(G, ((k < 2 ? qa : qb) & ~1) + (k & 1), tq, trq, tcq);
-#pragma unroll
-                for (int p = 0; p < C::NP; ++p)
-                    load_tile_panel(sK + k * C::TILE + p * C::PANEL, &tm_q, G, p, g, tq, trq, tcq, q_full);
-            }
+        int tqs[2], tcs[2];
+        for (int sl = 0; sl < 2; ++sl) {
+            int trx;
+            tile_coords(G, sl ? (hasB ? qb : qa) : qa, tqs[sl], trx, tcs[sl]);
         }
-        if (role_wait(q_full, 0, G.wait_ns, s_abort)) {
-            constexpr int CH = D / 8;                           // 16-byte chunks of a row
-            for (int i = tid; i < 128 * np * CH; i += C::THREADS) {
-                const int d = i / CH, ch = i - d * CH;
-                const int l = d < 128 ? grp_a[d] : grp_b[d - 128];
-                const int st = (d < 128 ? 0 : 2) + (l >> 7);     // staged tile
-                const int sr = l & 127, dr = d & 127, pn = ch >> 3, cc = ch & 7;
-                *reinterpret_cast<uint4*>(sQ + (d >> 7) * C::TILE + pn * C::PANEL + dr * 128 + ((cc ^ (dr & 7)) << 4)) =
-                    *reinterpret_cast<const uint4*>(sK + st * C::TILE + pn * C::PANEL + sr * 128 +
-                                                    ((cc ^ (sr & 7)) << 4));
+        for (int e = tid; e < 128 * np * CH; e += C::THREADS) {
+            const int d = e / CH, ch = e - d * CH;
+            const int sl = d >> 7, dr = d & 127;
+            const int l = (sl ? grp_b : grp_a)[dr];
+            const int hq = (l >> 7) * G.th + ((l & 127) >> TWL), wq = tcs[sl] * TW + (l & (TW - 1));
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (hq < G.H && wq < G.W) {
+                const int tl = (tqs[sl] * G.nTh + (l >> 7)) * G.nTw + tcs[sl];
+                const size_t qrow = io_row(G, g, tqs[sl], hq, wq, tl * 128 + (l & 127));
+                val = __ldg(reinterpret_cast<const uint4*>(qraw) + qrow * CH + ch);
             }
+            const int pn = ch >> 3, cc = ch & 7;
+            *reinterpret_cast<uint4*>(sQ + sl * C::TILE + pn * C::PANEL + dr * 128 + ((cc ^ (dr & 7)) << 4)) = val;
         }
         fence_proxy_async_smem();                               // generic smem writes -> tensor-core reads
         __syncthreads();
@@ -299,7 +294,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             } else {
                 prefetch_tmap(&tm_v);
             }
-            if (isK && !G.qsort) {                                  // else staged and gathered above
+            if (isK && !G.qsort) {                                  // else gathered above
                 mbar_arrive_expect_tx(q_full, C::TILE * (hasB ? 2 : 1));
                 int tqa, trqa, tcqa, tqb, trqb, tcqb;
                 tile_coords(G, qa, tqa, trqa, tcqa);
@@ -329,7 +324,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 ++iss;
             }
             // copies still in flight must land before the CTA exits
-            if (isK) mbar_wait(q_full, 0, G.drain_ns);
+            if (isK && !G.qsort) mbar_wait(q_full, 0, G.drain_ns);
             for (int j = max(0, iss - ST); j < iss; ++j) mbar_wait(&fullb[j % ST], (j / ST) & 1, G.drain_ns);
         }
       } else if (warp == C::WARP_MMA || warp == C::WARP_MMA + 1) {
@@ -349,7 +344,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
             const uint32_t sQa = smem_u32(sQ) + w * C::TILE, sKa = smem_u32(sK), sVa = smem_u32(sV);
             const uint32_t in_bit = MT_IN0 << w;
-            bool ok = role_wait(q_full, 0, G.wait_ns, s_abort);
+            bool ok = G.qsort || role_wait(q_full, 0, G.wait_ns, s_abort);     // grouped Q is already in place
             int cnt = 0;
             int qk_ahead = -1;                  // entry whose QK went out with the previous PV group
             auto issue_qk = [&](int jj) {
@@ -436,19 +431,30 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t colS = col_s(w), colO = col_o(w);
         const bool active = w == 0 || hasB;
-        // this thread's query: row `row` of tile qa / qb, or the pair row of
+        // this thread's query: row `row` of tile qa / qb, or the strip row of
         // its group slot (radius-sorted groups)
         int qt = w ? qb : qa, qrow = row;
+        bool grp_ok = true;
         if (G.qsort && active) {
-            const int l = (w ? grp_b : grp_a)[row];
-            qt = (qt & ~1) + (l >> 7);
+            // strip row l: row l & 127 of the tile in tile row l >> 7 of the
+            // slot's tile column and frame.  The group section is caller
+            // memory: a row past the strip is recorded and the slot left empty.
+            int l = (w ? grp_b : grp_a)[row];
+            if (l >= 128 * G.nTh) {
+                atomicOr(&g_tra_error, TRA_ERRBIT_CHECK);
+                l = 0;
+                grp_ok = false;
+            }
+            int t0, tr0, tc0;
+            tile_coords(G, qt, t0, tr0, tc0);
+            qt = (t0 * G.nTh + (l >> 7)) * G.nTw + tc0;
             qrow = l & 127;
         }
         int tq, trq, tcq;
         tile_coords(G, active ? qt : qa, tq, trq, tcq);
         const int hq = trq * G.th + (qrow >> TWL);
         const int wq = tcq * TW + (qrow & (TW - 1));
-        const bool qvalid = active && hq < G.H && wq < G.W;
+        const bool qvalid = active && grp_ok && hq < G.H && wq < G.W;
         const int rq = qvalid ? reinterpret_cast<const int32_t*>(mask + G.off_radius)[kbase + qt * 128 + qrow] : -1;
         uint16_t* my_tab = s_tab + w * (G.rte + 1) * 128;
         for (int dl = 0; dl <= G.rte; ++dl)

@@ -6,44 +6,57 @@
 // "Noyaux CUDA Fusionnes" (distance computation, radius comparison, block
 // pruning and token voting fused into one kernel that emits a block-sparse
 // mask).  Token voting is read as an OR vote: a key tile is listed for a query
-// tile iff some retained token pair falls in it, so skipping unlisted tiles
+// set iff some retained token pair falls in it, so skipping unlisted tiles
 // never changes the attention output.
 //
-// One CTA per (query tile, head), one thread per tile row (token).
+// One CTA per (strip, head), one thread per row.  A strip is U tiles: with
+// radius-sorted query groups (a scheduling choice of this library) the U =
+// nTh tiles of one tile column of one frame, otherwise a single tile.
+//   0. The half-widths s(r, |dt|) = floor(r * gamma^|dt| + 1e-9) of every r in
+//      [0, r_cap] go into a shared table when it is small (the same fp64 rule,
+//      evaluated once per entry instead of once per search probe).
 //   1. Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))), y = a*H + b in fp64 and
 //      the ceiling of e^y decided exactly.
 //   2. r = the smallest r in [0, r_cap] whose clipped neighbourhood count
 //      reaches Bhat (binary search; the count is monotone in r).
-//   3. Per frame distance |dt|: every query's neighbourhood is a rectangle of
-//      key tiles that contains the query tile's own tile position, so for a
-//      key tile row the union over the tile's queries is one interval of tile
-//      columns (warp min/max reductions), and the "full" tiles (every valid
-//      pair retained) are the intersection of per-query rectangles.
-//   4. The active tiles of the frames within Rt' are written in ascending
-//      tile order after a block-wide prefix sum over (frame, tile row).
-// With radius-sorted query groups (a scheduling choice of this library) each
-// CTA first finds the radii of both tiles of its pair (2p, 2p+1: side by side
-// in one tile row), orders the pair's 256 rows by (radius, row), and then
-// speaks for the 128 queries of its own group instead of its own tile's rows;
-// step 3 still holds because every member's rectangle contains its own tile
-// column, one of two adjacent columns of the same tile row.
+//   3. Groups: with query groups the strip's 128*U rows are ordered by
+//      (radius, strip row), pad rows first (each warp sorts its 32 keys with
+//      shuffles; a key's rank adds its position in its own warp to a binary
+//      search in every other warp's sorted keys); warpgroup u then speaks for
+//      the u-th block of 128, the group of the strip's tile in tile row u.
+//      Without groups warpgroup 0 speaks for its tile's own rows.
+//   4. Per group and frame distance |dt|: every member's neighbourhood is a
+//      rectangle of key tiles that contains the member's own tile column --
+//      the strip's column -- so for a key tile row the union over the members
+//      is one interval of tile columns (warp min/max reductions), and the
+//      "full" tiles (every valid pair retained) are the intersection of the
+//      members' rectangles.
+//   5. Each group's active tiles of the frames within Rt' are written in
+//      ascending tile order after a prefix sum over (frame, tile row).
 #pragma once
 #include "exact_budget.cuh"
 #include "tra_common.cuh"
 
 namespace tra {
 
+// the spatial half-width at radius r and frame distance dl: from the shared
+// table when the plan has one, else evaluated
+__device__ __forceinline__ int hw_at(const Geom& G, const uint16_t* tab, int r, int dl)
+{
+    return tab ? (int)tab[dl * (G.r_cap + 1) + r] : halfwidth(r, G.g[dl]);
+}
+
 // clipped neighbourhood count c(r) of the query at (t, h, w): per frame the
 // Chebyshev square is a clipped rectangle; the disk sums, key row by key row,
 // the clipped width 2*isqrt(s^2 - dh^2) + 1
 template <bool DISK>
-__device__ __forceinline__ long long nbr_count(const Geom& G, int t, int h, int w, int r)
+__device__ __forceinline__ long long nbr_count(const Geom& G, const uint16_t* tab, int t, int h, int w, int r)
 {
     long long c = 0;
     for (int dl = 0; dl <= G.rte; ++dl) {
         const int m = (t + dl < G.T ? 1 : 0) + (dl > 0 && t - dl >= 0 ? 1 : 0);
         if (m == 0) break;                         // farther frames are out of the grid too
-        const int s = halfwidth(r, G.g[dl]);
+        const int s = hw_at(G, tab, r, dl);
         if constexpr (DISK) {
             // key rows h - k (k <= up) and h + k (k <= dn) share the half-width
             // isqrt(s^2 - k^2)
@@ -77,7 +90,8 @@ __device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
 // r = the smallest r in [0, r_cap] whose neighbourhood count reaches bh (the
 // count is monotone in r; r_cap when none does); c = that count.
 template <bool DISK>
-__device__ __forceinline__ int find_radius(const Geom& G, int t, int h, int w, long long bh, long long& c)
+__device__ __forceinline__ int find_radius(const Geom& G, const uint16_t* tab, int t, int h, int w, long long bh,
+                                           long long& c)
 {
     int lo = 0, hi = G.r_cap;
     if constexpr (DISK) {
@@ -86,126 +100,154 @@ __device__ __forceinline__ int find_radius(const Geom& G, int t, int h, int w, l
         // that bracket reaches the budget, else the rest up to r_cap
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (nbr_count<false>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+            if (nbr_count<false>(G, tab, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
         }
         const int r2 = min(G.r_cap, 2 * lo + 2);
-        if (nbr_count<true>(G, t, h, w, r2) >= bh) hi = r2;
+        if (nbr_count<true>(G, tab, t, h, w, r2) >= bh) hi = r2;
         else { lo = min(r2 + 1, G.r_cap); hi = G.r_cap; }
     }
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (nbr_count<DISK>(G, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+        if (nbr_count<DISK>(G, tab, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
     }
-    c = nbr_count<DISK>(G, t, h, w, lo);
+    c = nbr_count<DISK>(G, tab, t, h, w, lo);
     return lo;
 }
 
+// Rows of a strip: 128 per tile, at most TRA_MAX_STRIP_TILES tiles.
+constexpr int MASK_MAX_ROWS = 128 * TRA_MAX_STRIP_TILES;
+
 // Dynamic shared memory of the mask kernel, sized from the plan so that small
-// reaches keep many CTAs resident: per (frame distance, tile row) the active
-// column interval [lo, hi] and the disk's full-column bits, and per list row
-// (frame, tile row) its length.
-// With radius-sorted groups it also holds the pair's 256 counts, radii and
-// the group order.
-__host__ __device__ inline int mask_smem_bytes(int rte, int nTh, bool qsort)
+// reaches keep many CTAs resident.  In order: the half-width table (uint16,
+// when the plan has one), and per group u < U the column interval [lo, hi]
+// and the disk's full-column bits of every (frame distance, tile row), the
+// length of every list row (frame, tile row).
+__host__ __device__ inline int mask_tab_bytes(int rte, int r_cap, bool tab)
 {
-    return (qsort ? 256 * (8 + 4 + 4) : 0) + (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
+    return tab ? ((rte + 1) * (r_cap + 1) * 2 + 15) & ~15 : 0;
+}
+__host__ __device__ inline int mask_smem_bytes(int rte, int nTh, int r_cap, bool tab, int U)
+{
+    return mask_tab_bytes(rte, r_cap, tab) + U * (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
 }
 
 template <bool DISK, bool QS>
-__global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
-                                                          uint8_t* __restrict__ mask)
+__global__ void __launch_bounds__(MASK_MAX_ROWS) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
+                                                                    uint8_t* __restrict__ mask)
 {
-    extern __shared__ __align__(16) long long mask_smem[];
+    extern __shared__ __align__(16) uint8_t mask_dyn[];
+    const int U = QS ? G.nTh : 1;                                 // tiles (and groups) of this CTA
     const int RS = G.nTh;                                         // stride of one frame distance
-    long long* s_qc = mask_smem;                                  // QS: [256] counts of the pair's rows
-    int* s_qr = reinterpret_cast<int*>(s_qc + (QS ? 256 : 0));    // QS: [256] radii of the pair's rows
-    int* s_qp = s_qr + (QS ? 256 : 0);                            // QS: [256] pair rows in group order
-    int* s_lo = s_qp + (QS ? 256 : 0);                            // [rte + 1][nTh]
+    const uint16_t* tab = G.hw_tab ? reinterpret_cast<const uint16_t*>(mask_dyn) : nullptr;
+    int* grp_base = reinterpret_cast<int*>(mask_dyn + mask_tab_bytes(G.rte, G.r_cap, G.hw_tab != 0));
+    const int GS = 3 * (G.rte + 1) * RS + (2 * G.rte + 1) * RS;   // ints per group
+    constexpr int QR = QS ? MASK_MAX_ROWS : 1;
+    __shared__ int s_key[QR];                  // QS: warp-sorted keys (radius + 1) << 10 | strip row
+    __shared__ int s_order[QR];                // QS: strip rows in group order
+    __shared__ int s_rad[QR];                  // QS: radius of every strip row
+    __shared__ long long s_cnt[QR];            // QS: its count c(r)
+    __shared__ int s_full[TRA_MAX_STRIP_TILES][TRA_MAX_RT_EFF + 1][4];
+    __shared__ long long s_pairs[MASK_MAX_ROWS / 32];
+    __shared__ int s_warp[MASK_MAX_ROWS / 32];
+
+    const int g = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int u = tid >> 7, i = tid & 127;                        // group (warpgroup) and slot
+    // the strip: frame t, tile column tc (QS); or tile blockIdx.x
+    int t, tr0, tc;
+    if (QS) {
+        t = blockIdx.x / G.nTw;
+        tc = blockIdx.x - t * G.nTw;
+        tr0 = 0;
+    } else {
+        tile_coords(G, blockIdx.x, t, tr0, tc);
+    }
+    auto strip_tile = [&](int uu) { return (t * G.nTh + tr0 + uu) * G.nTw + tc; };
+
+    if (tab) {
+        const int n = (G.rte + 1) * (G.r_cap + 1);
+        uint16_t* wtab = reinterpret_cast<uint16_t*>(mask_dyn);
+        for (int e = tid; e < n; e += blockDim.x) {
+            const int dl = e / (G.r_cap + 1);
+            wtab[e] = (uint16_t)halfwidth(e - dl * (G.r_cap + 1), G.g[dl]);
+        }
+    }
+    int* s_lo = grp_base + u * GS;                                // [rte + 1][nTh]
     int* s_hi = s_lo + (G.rte + 1) * RS;                          // [rte + 1][nTh]
     uint32_t* s_fullbits = reinterpret_cast<uint32_t*>(s_hi + (G.rte + 1) * RS);   // disk: full tile columns
     int* s_len = reinterpret_cast<int*>(s_fullbits + (G.rte + 1) * RS);            // [(2 rte + 1) nTh]
-    __shared__ int s_full[TRA_MAX_RT_EFF + 1][4];
-    __shared__ long long s_pairs[4];
-    __shared__ int s_warp[4];
-
-    const int tile = blockIdx.x, g = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int t, trq, tcq;
-    tile_coords(G, tile, t, trq, tcq);
-
-    for (int i = tid; i < (G.rte + 1) * RS; i += 128) {
-        s_lo[i] = 0x7fffffff;
-        s_hi[i] = -1;
-        s_fullbits[i] = 0xffffffffu;
+    for (int e = i; e < (G.rte + 1) * RS; e += 128) {
+        s_lo[e] = 0x7fffffff;
+        s_hi[e] = -1;
+        s_fullbits[e] = 0xffffffffu;
     }
-    if (tid < G.rte + 1) {
-        s_full[tid][0] = -0x7fffffff; s_full[tid][1] = 0x7fffffff;
-        s_full[tid][2] = -0x7fffffff; s_full[tid][3] = 0x7fffffff;
+    if (i < G.rte + 1) {
+        s_full[u][i][0] = -0x7fffffff; s_full[u][i][1] = 0x7fffffff;
+        s_full[u][i][2] = -0x7fffffff; s_full[u][i][3] = 0x7fffffff;
     }
+    __syncthreads();
 
-    // ---- budget and radius of the query this thread speaks for: its own row
-    // of the tile, or (QS) a slot of the tile's radius-sorted group
-    int h, w, r = -1;
-    bool valid;
+    // ---- budget and radius of strip row `tid` (tile u of the strip, row i)
+    int h = (tr0 + u) * G.th + (i >> G.tw_log2);
+    int w = tc * G.tw + (i & (G.tw - 1));
+    bool valid = h < G.H && w < G.W;
+    int r = -1;
     long long c = 0;
-    if constexpr (!QS) {
-        h = trq * G.th + (tid >> G.tw_log2);
-        w = tcq * G.tw + (tid & (G.tw - 1));
-        valid = h < G.H && w < G.W;
-        if (valid) r = find_radius<DISK>(G, t, h, w, budget_hat(G, Hent[io_row(G, g, t, h, w, tile * 128 + tid)]), c);
-        reinterpret_cast<int32_t*>(mask + G.off_radius)[(size_t)g * G.N_pad + (size_t)tile * 128 + tid] = r;
-    } else {
-        // both tiles of the pair (tiles 2p, 2p+1 side by side in one tile row)
-        const int pb = tile & ~1;
-        for (int k = 0; k < 2; ++k) {
-            const int hk = trq * G.th + (tid >> G.tw_log2);
-            const int wk = (tcq - (tile & 1) + k) * G.tw + (tid & (G.tw - 1));
-            int rk = -1;
-            long long ck = 0;
-            if (hk < G.H && wk < G.W)
-                rk = find_radius<DISK>(G, t, hk, wk, budget_hat(G, Hent[io_row(G, g, t, hk, wk, (pb + k) * 128 + tid)]), ck);
-            s_qr[k * 128 + tid] = rk;
-            s_qc[k * 128 + tid] = ck;
-            if (pb + k == tile)
-                reinterpret_cast<int32_t*>(mask + G.off_radius)[(size_t)g * G.N_pad + (size_t)tile * 128 + tid] = rk;
-        }
-        __syncthreads();
-        // order the pair's rows by (radius, row); pad rows (radius -1) first
-        for (int k = 0; k < 2; ++k) {
-            const int l = k * 128 + tid, rl = s_qr[l];
-            int rank = 0;
-            for (int j = 0; j < 256; ++j) {
-                const int rj = s_qr[j];
-                rank += (rj < rl || (rj == rl && j < l)) ? 1 : 0;
-            }
-            s_qp[rank] = l;
-        }
-        __syncthreads();
-        const int l = s_qp[(tile & 1) * 128 + tid];
-        h = trq * G.th + ((l & 127) >> G.tw_log2);
-        w = (tcq - (tile & 1) + (l >> 7)) * G.tw + (l & (G.tw - 1));
-        valid = h < G.H && w < G.W;
-        r = s_qr[l];
-        c = s_qc[l];
-        mask[G.off_group + ((size_t)g * G.nQ + tile) * 128 + tid] = (uint8_t)l;
-    }
+    if (valid) r = find_radius<DISK>(G, tab, t, h, w, budget_hat(G, Hent[io_row(G, g, t, h, w, strip_tile(u) * 128 + i)]), c);
+    reinterpret_cast<int32_t*>(mask + G.off_radius)[(size_t)g * G.N_pad + (size_t)strip_tile(u) * 128 + i] = r;
 
-    // ---- retained pairs of the tile
+    if constexpr (QS) {
+        // ---- order the strip's rows by (radius, row), pads (radius -1) first
+        s_rad[tid] = r;
+        s_cnt[tid] = c;
+        int key = ((r + 1) << 10) | tid;
+        for (int k = 2; k <= 32; k <<= 1)
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                const int other = __shfl_xor_sync(0xffffffffu, key, j);
+                const bool up = (lane & k) == 0, low = (lane & j) == 0;
+                key = (low == up) ? min(key, other) : max(key, other);
+            }
+        s_key[tid] = key;
+        __syncthreads();
+        int rank = lane;
+        for (int ow = 0; ow < 4 * U; ++ow) {
+            if (ow == warp) continue;
+            const int* sk = s_key + ow * 32;
+            int lo = 0;                                           // keys of warp ow below `key`
+#pragma unroll
+            for (int step = 16; step > 0; step >>= 1)
+                if (sk[lo + step - 1] < key) lo += step;
+            lo += sk[lo] < key ? 1 : 0;
+            rank += lo;
+        }
+        s_order[rank] = key & 1023;
+        __syncthreads();
+        const int l = s_order[tid];                               // the strip row group u's slot i speaks for
+        h = (l >> 7) * G.th + ((l & 127) >> G.tw_log2);
+        w = tc * G.tw + (l & (G.tw - 1));
+        valid = h < G.H && w < G.W;
+        r = s_rad[l];
+        c = s_cnt[l];
+        reinterpret_cast<uint16_t*>(mask + G.off_group)[((size_t)g * G.nQ + strip_tile(u)) * 128 + i] = (uint16_t)l;
+    }
+    const int tile = strip_tile(u);                               // this group's mask slot
+
+    // ---- retained pairs of the group
     long long cs = c;
     for (int o = 16; o > 0; o >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
     if (lane == 0) s_pairs[warp] = cs;
     __syncthreads();
-    if (tid == 0)
+    if (i == 0)
         reinterpret_cast<long long*>(mask + G.off_pairs)[(size_t)g * G.nQ + tile] =
-            s_pairs[0] + s_pairs[1] + s_pairs[2] + s_pairs[3];
+            s_pairs[4 * u] + s_pairs[4 * u + 1] + s_pairs[4 * u + 2] + s_pairs[4 * u + 3];
 
     // ---- per frame distance: active tile-column interval per tile row, full rectangle
     for (int dl = 0; dl <= G.rte; ++dl) {
         if (!(t + dl < G.T || t - dl >= 0)) break;    // uniform over the CTA
         int rl = 0x7fffffff, rh = -1, cl = 0, ch = -1;
         int frl = -0x7fffffff, frh = 0x7fffffff, fcl = -0x7fffffff, fch = 0x7fffffff;
+        const int s = valid ? hw_at(G, tab, r, dl) : 0;
         if (valid) {
-            const int s = halfwidth(r, G.g[dl]);
             rl = max(0, h - s) >> G.th_log2;
             rh = min(G.H - 1, h + s) >> G.th_log2;
             cl = max(0, w - s) >> G.tw_log2;
@@ -220,8 +262,8 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         fcl = __reduce_max_sync(0xffffffffu, fcl);
         fch = __reduce_min_sync(0xffffffffu, fch);
         if (lane == 0) {
-            atomicMax(&s_full[dl][0], frl); atomicMin(&s_full[dl][1], frh);
-            atomicMax(&s_full[dl][2], fcl); atomicMin(&s_full[dl][3], fch);
+            atomicMax(&s_full[u][dl][0], frl); atomicMin(&s_full[u][dl][1], frh);
+            atomicMax(&s_full[u][dl][2], fcl); atomicMin(&s_full[u][dl][3], fch);
         }
         const int r_lo = __reduce_min_sync(0xffffffffu, rl);
         const int r_hi = __reduce_max_sync(0xffffffffu, rh);
@@ -230,10 +272,10 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
             int c_lo = cl, c_hi = ch;
             if (DISK && in) {
                 // the disk is widest on the tile row's key row nearest to h
-                const int s = min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP);
+                const int sc = min(s, TRA_DISK_S_CLAMP);
                 const int k0 = tr * G.th, k1 = min(G.H - 1, k0 + G.th - 1);
                 const int dh = h < k0 ? k0 - h : (h > k1 ? h - k1 : 0);
-                const int half = isqrt_floor(s * s - dh * dh);
+                const int half = isqrt_floor(sc * sc - dh * dh);
                 c_lo = max(0, w - half) >> G.tw_log2;
                 c_hi = min(G.W - 1, w + half) >> G.tw_log2;
             }
@@ -252,18 +294,18 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     if constexpr (DISK) {
         for (int dl = 0; dl <= G.rte; ++dl) {
             if (!(t + dl < G.T || t - dl >= 0)) break;
-            const int s = valid ? min(halfwidth(r, G.g[dl]), TRA_DISK_S_CLAMP) : 0;
+            const int s = valid ? min(hw_at(G, tab, r, dl), TRA_DISK_S_CLAMP) : 0;
             for (int tr = 0; tr < G.nTh; ++tr) {
                 const int lo = s_lo[dl * RS + tr], hi = s_hi[dl * RS + tr];
                 if (hi < 0) continue;
                 const int k0 = tr * G.th, k1 = min(G.H - 1, k0 + G.th - 1);
                 const int dh = max(abs(h - k0), abs(h - k1));
                 uint32_t bits = 0;
-                for (int tc = lo; tc <= hi; ++tc) {
-                    const int j0 = tc * G.tw, j1 = min(G.W - 1, j0 + G.tw - 1);
+                for (int tcol = lo; tcol <= hi; ++tcol) {
+                    const int j0 = tcol * G.tw, j1 = min(G.W - 1, j0 + G.tw - 1);
                     const int dw = max(abs(w - j0), abs(w - j1));
                     const bool in = !valid || (long long)dh * dh + (long long)dw * dw <= (long long)s * s;
-                    if (__all_sync(0xffffffffu, in)) bits |= 1u << tc;
+                    if (__all_sync(0xffffffffu, in)) bits |= 1u << tcol;
                 }
                 if (lane == 0) atomicAnd(&s_fullbits[dl * RS + tr], bits | ~(((2u << hi) - 1u) ^ ((1u << lo) - 1u)));
             }
@@ -271,19 +313,19 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
         __syncthreads();
     }
 
-    // ---- list rows (frame, tile row) in ascending tile order; block prefix sum
+    // ---- list rows (frame, tile row) in ascending tile order; prefix sum over the group
     const int t0 = max(0, t - G.rte), t1 = min(G.T - 1, t + G.rte);
     const int R = (t1 - t0 + 1) * G.nTh;
-    for (int i = tid; i < R; i += 128) {
-        const int f = i / G.nTh, tr = i - f * G.nTh;
+    for (int e = i; e < R; e += 128) {
+        const int f = e / G.nTh, tr = e - f * G.nTh;
         const int dl = abs(t0 + f - t);
-        s_len[i] = s_hi[dl * RS + tr] >= 0 ? s_hi[dl * RS + tr] - s_lo[dl * RS + tr] + 1 : 0;
+        s_len[e] = s_hi[dl * RS + tr] >= 0 ? s_hi[dl * RS + tr] - s_lo[dl * RS + tr] + 1 : 0;
     }
     __syncthreads();
     const int per = (R + 127) >> 7;
-    const int beg = min(R, tid * per), end = min(R, beg + per);
+    const int beg = min(R, i * per), end = min(R, beg + per);
     int local = 0;
-    for (int i = beg; i < end; ++i) local += s_len[i];
+    for (int e = beg; e < end; ++e) local += s_len[e];
     int incl = local;
     for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -292,24 +334,24 @@ __global__ void __launch_bounds__(128) radius_mask_kernel(const Geom G, const fl
     if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
     int off = incl - local;
-    for (int k = 0; k < warp; ++k) off += s_warp[k];
+    for (int k = 4 * u; k < warp; ++k) off += s_warp[k];
     uint16_t* list = reinterpret_cast<uint16_t*>(mask + G.off_list) + ((size_t)g * G.nQ + tile) * G.list_cap;
-    for (int i = beg; i < end; ++i) {
-        const int f = i / G.nTh, tr = i - f * G.nTh;
+    for (int e = beg; e < end; ++e) {
+        const int f = e / G.nTh, tr = e - f * G.nTh;
         const int dl = abs(t0 + f - t);
         const int lo = s_lo[dl * RS + tr], hi = s_hi[dl * RS + tr];
-        const bool row_full = s_full[dl][0] <= tr && tr <= s_full[dl][1];
+        const bool row_full = s_full[u][dl][0] <= tr && tr <= s_full[u][dl][1];
         const uint32_t fbits = s_fullbits[dl * RS + tr];
         const int base = ((t0 + f) * G.nTh + tr) * G.nTw;
-        for (int tc = lo; tc <= hi; ++tc) {
-            const bool full = DISK ? ((fbits >> tc) & 1u) != 0
-                                     : (row_full && s_full[dl][2] <= tc && tc <= s_full[dl][3]);
-            list[off++] = (uint16_t)((base + tc) | (full ? 0x8000 : 0));
+        for (int tcol = lo; tcol <= hi; ++tcol) {
+            const bool full = DISK ? ((fbits >> tcol) & 1u) != 0
+                                   : (row_full && s_full[u][dl][2] <= tcol && tcol <= s_full[u][dl][3]);
+            list[off++] = (uint16_t)((base + tcol) | (full ? 0x8000 : 0));
         }
     }
-    if (tid == 0)
+    if (i == 0)
         reinterpret_cast<int32_t*>(mask + G.off_count)[(size_t)g * G.nQ + tile] =
-            s_warp[0] + s_warp[1] + s_warp[2] + s_warp[3];
+            s_warp[4 * u] + s_warp[4 * u + 1] + s_warp[4 * u + 2] + s_warp[4 * u + 3];
 }
 
 }  // namespace tra

@@ -91,7 +91,7 @@ constexpr int kMaxSmem = 232448;
 
 template <int D, int TWL, bool OB, bool DISK>
 tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                         const uint8_t* mask, void* out, cudaStream_t st)
+                         const uint8_t* mask, void* out, const void* qraw, cudaStream_t st)
 {
     using C = tra::AttnCfg<D>;
     auto kern = tra::attention_kernel<D, TWL, OB, DISK>;
@@ -101,7 +101,7 @@ tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtenso
     // two query tiles per CTA; with radius-sorted groups, the same slot of
     // frames 2f and 2f + 1
     const int ctas = G.qsort ? (G.T + 1) / 2 * G.tiles_per_frame : (G.nQ + 1) / 2;
-    kern<<<dim3(ctas, G.G), C::THREADS, smem, st>>>(q, k, v, G, mask, out);
+    kern<<<dim3(ctas, G.G), C::THREADS, smem, st>>>(q, k, v, G, mask, out, qraw);
     return launch_status();
 }
 
@@ -183,17 +183,22 @@ extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void
     if (!plan || !Hent || !mask || !aligned(Hent, 4) || !aligned(mask, 256)) return TRA_ERR_INVALID_ARG;
     if (mask_bytes < plan->mask_bytes) return TRA_ERR_WORKSPACE;
     const tra::Geom& G = plan->geom;
-    const dim3 grid(G.nQ, G.G);
-    const int smem = tra::mask_smem_bytes(G.rte, G.nTh, G.qsort != 0);   // at most 44.8 KB
+    // one CTA per tile-column strip (query groups) or per tile
+    const int U = G.qsort ? G.nTh : 1;
+    const dim3 grid(G.qsort ? G.T * G.nTw : G.nQ, G.G);
+    const int smem = tra::mask_smem_bytes(G.rte, G.nTh, G.r_cap, G.hw_tab != 0, U);
+    if (smem > kMaxSmem - 16 * 1024) return TRA_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* m = (uint8_t*)mask;
-    if (G.qsort) {
-        if (G.disk) tra::radius_mask_kernel<true, true><<<grid, 128, smem, st>>>(G, Hent, m);
-        else tra::radius_mask_kernel<false, true><<<grid, 128, smem, st>>>(G, Hent, m);
-    } else {
-        if (G.disk) tra::radius_mask_kernel<true, false><<<grid, 128, smem, st>>>(G, Hent, m);
-        else tra::radius_mask_kernel<false, false><<<grid, 128, smem, st>>>(G, Hent, m);
-    }
+    auto go = [&](auto kern) -> bool {
+        if (smem > 48 * 1024 && !set_smem(kern, smem)) return false;
+        kern<<<grid, 128 * U, smem, st>>>(G, Hent, m);
+        return true;
+    };
+    bool ok;
+    if (G.qsort) ok = G.disk ? go(tra::radius_mask_kernel<true, true>) : go(tra::radius_mask_kernel<false, true>);
+    else ok = G.disk ? go(tra::radius_mask_kernel<true, false>) : go(tra::radius_mask_kernel<false, false>);
+    if (!ok) return TRA_ERR_CUDA;
     return launch_status();
 }
 
@@ -201,27 +206,27 @@ namespace {
 
 template <int D, int TWL>
 tra_status attention_variant(const tra::Geom& G, bool ob, bool disk, const CUtensorMap& q, const CUtensorMap& k,
-                             const CUtensorMap& v, const uint8_t* m, void* out, cudaStream_t st)
+                             const CUtensorMap& v, const uint8_t* m, void* out, const void* qr, cudaStream_t st)
 {
-    if (ob) return disk ? run_attention<D, TWL, true, true>(G, q, k, v, m, out, st)
-                        : run_attention<D, TWL, true, false>(G, q, k, v, m, out, st);
-    return disk ? run_attention<D, TWL, false, true>(G, q, k, v, m, out, st)
-                : run_attention<D, TWL, false, false>(G, q, k, v, m, out, st);
+    if (ob) return disk ? run_attention<D, TWL, true, true>(G, q, k, v, m, out, qr, st)
+                        : run_attention<D, TWL, true, false>(G, q, k, v, m, out, qr, st);
+    return disk ? run_attention<D, TWL, false, true>(G, q, k, v, m, out, qr, st)
+                : run_attention<D, TWL, false, false>(G, q, k, v, m, out, qr, st);
 }
 
 // kernel instance by (head dim, tile width, output type, spatial metric)
 tra_status dispatch_attention(const tra::Geom& G, bool ob, bool disk, const CUtensorMap& q, const CUtensorMap& k,
-                              const CUtensorMap& v, const uint8_t* m, void* out, cudaStream_t st)
+                              const CUtensorMap& v, const uint8_t* m, void* out, const void* qr, cudaStream_t st)
 {
     switch (G.D * 100 + G.tw_log2) {
-        case 6402: return attention_variant<64, 2>(G, ob, disk, q, k, v, m, out, st);
-        case 6403: return attention_variant<64, 3>(G, ob, disk, q, k, v, m, out, st);
-        case 6404: return attention_variant<64, 4>(G, ob, disk, q, k, v, m, out, st);
-        case 6405: return attention_variant<64, 5>(G, ob, disk, q, k, v, m, out, st);
-        case 12802: return attention_variant<128, 2>(G, ob, disk, q, k, v, m, out, st);
-        case 12803: return attention_variant<128, 3>(G, ob, disk, q, k, v, m, out, st);
-        case 12804: return attention_variant<128, 4>(G, ob, disk, q, k, v, m, out, st);
-        case 12805: return attention_variant<128, 5>(G, ob, disk, q, k, v, m, out, st);
+        case 6402: return attention_variant<64, 2>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 6403: return attention_variant<64, 3>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 6404: return attention_variant<64, 4>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 6405: return attention_variant<64, 5>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 12802: return attention_variant<128, 2>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 12803: return attention_variant<128, 3>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 12804: return attention_variant<128, 4>(G, ob, disk, q, k, v, m, out, qr, st);
+        case 12805: return attention_variant<128, 5>(G, ob, disk, q, k, v, m, out, qr, st);
     }
     return TRA_ERR_UNSUPPORTED;
 }
@@ -242,7 +247,7 @@ extern "C" tra_status tra_attention(tra_plan plan, const void* q, const void* k,
     const uint8_t* m = (const uint8_t*)mask;
     const bool ob = (plan->flags & TRA_FLAG_OUT_BF16) != 0;
     const bool disk = G.disk != 0;
-    return dispatch_attention(G, ob, disk, mq, mk, mv, m, out, st);
+    return dispatch_attention(G, ob, disk, mq, mk, mv, m, out, q, st);
 }
 
 extern "C" tra_status tra_calibrate_topk(tra_plan plan, const void* q, const void* k, double mass,

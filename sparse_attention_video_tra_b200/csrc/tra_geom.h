@@ -9,6 +9,8 @@
 #define TRA_MAX_R_CAP (1 << 20)
 #define TRA_MAX_LIST_CAP 2048         // key tiles listed per query tile
 #define TRA_MAX_HW 256                // largest H and W (half-widths kept as bytes)
+#define TRA_MAX_STRIP_TILES 4         // tile rows per frame with radius-sorted query groups
+#define TRA_MAX_HW_TAB 8192           // half-width table entries (Rt'+1)(r_cap+1) kept in shared memory
 #define TRA_ERRBIT_TIMEOUT 1u
 #define TRA_ERRBIT_CHECK 2u
 
@@ -29,7 +31,8 @@ struct Geom {
     unsigned long long drain_ns;     // limit of the waits that drain in-flight copies
     int natural;                     // q/k/v/out/entropies in natural token order (4-D TMA boxes)
     int disk;                        // spatial test dh^2 + dw^2 <= s^2 instead of the Chebyshev square
-    int qsort;                       // radius-sorted query groups of tile pairs
+    int qsort;                       // radius-sorted query groups of tile-column strips
+    int hw_tab;                      // the mask kernel tabulates s(r, |dt|) for r <= r_cap
 };
 
 }  // namespace tra

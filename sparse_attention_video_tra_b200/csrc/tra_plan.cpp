@@ -125,10 +125,11 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     G.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     G.wait_ns = (flags & TRA_FLAG_DEBUG_NO_WAIT) ? 0ull : 2000000000ull;
     G.natural = (flags & TRA_FLAG_NATURAL) ? 1 : 0;
-    // radius-sorted groups pair tiles 2p and 2p+1, which sit side by side in
-    // one tile row only when a frame has an even number of tile columns
+    // radius-sorted groups sort the rows of a tile-column strip (one tile
+    // column of one frame, nTh tiles) in one CTA of 128 * nTh threads
     G.qsort = (flags & TRA_FLAG_QSORT) ? 1 : 0;
-    if (G.qsort && (G.nTw & 1)) return TRA_ERR_UNSUPPORTED;
+    if (G.qsort && G.nTh > TRA_MAX_STRIP_TILES) return TRA_ERR_UNSUPPORTED;
+    G.hw_tab = (long long)(rte + 1) * (G.r_cap + 1) <= TRA_MAX_HW_TAB ? 1 : 0;
     G.drain_ns = 2000000000ull;
 
     // mask buffer layout
@@ -138,7 +139,7 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     G.off_pairs = (long long)off;   off = align256(off + sizeof(long long) * (size_t)heads * nQ);
     G.off_list = (long long)off;    off = align256(off + sizeof(uint16_t) * (size_t)heads * nQ * G.list_cap);
     G.off_group = 0;
-    if (G.qsort) { G.off_group = (long long)off; off = align256(off + (size_t)heads * nQ * 128); }
+    if (G.qsort) { G.off_group = (long long)off; off = align256(off + sizeof(uint16_t) * (size_t)heads * nQ * 128); }
 
     tra_plan_s* p = new (std::nothrow) tra_plan_s;
     if (!p) return TRA_ERR_INVALID_ARG;

@@ -162,14 +162,16 @@ def test_workload_tiles_match_the_documented_choice():
     assert (portrait.tile_h, portrait.tile_w) == (8, 16) and portrait.N_pad == 2 * 3840
 
 
-def test_qsort_needs_an_even_number_of_tile_columns():
-    # (1,16,8) tiles at 45x80: 10 columns, accepted, with a group section
+def test_qsort_needs_at_most_four_tile_rows():
+    # (1,16,8) tiles at 45x80: 3 tile rows, accepted, with a uint16 group section
     p = tra.Plan(21, 45, 80, 2, 128, 1.0, 0.0, 0.8, 6, 8, flags=tra.TRA_FLAG_QSORT)
     i = p.info
     assert i.off_group % 256 == 0 and i.off_group >= i.off_list + 2 * i.heads * i.n_tiles * i.list_cap
-    assert i.mask_bytes >= i.off_group + i.heads * i.n_tiles * 128
+    assert i.mask_bytes >= i.off_group + 2 * i.heads * i.n_tiles * 128
     assert tra.Plan(21, 45, 80, 2, 128, 1.0, 0.0, 0.8, 6, 8).info.off_group == 0
-    # (1,32,4) tiles at 30x52: 13 columns, rejected
+    # (1,32,4) tiles at 30x52: one tile row, accepted (the groups are the tiles)
+    tra.Plan(21, 30, 52, 2, 128, 1.0, 0.0, 0.8, 6, 8, flags=tra.TRA_FLAG_QSORT).close()
+    # 200 rows: 13 tile rows of 16, rejected
     with pytest.raises(tra.TraError) as e:
-        tra.tra_plan_create(21, 30, 52, 2, 128, 1.0, 0.0, 0.8, 6, 8, flags=tra.TRA_FLAG_QSORT)
+        tra.tra_plan_create(2, 200, 200, 2, 128, 1.0, 0.0, 0.8, 1, 8, flags=tra.TRA_FLAG_QSORT)
     assert e.value.status == 2

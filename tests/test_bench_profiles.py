@@ -45,15 +45,20 @@ def test_stale_or_missing_summary_reports_no_traffic(tmp_path, monkeypatch):
 
 
 def test_query_group_default_follows_the_plan():
-    """--qsort auto turns radius-sorted query groups on exactly where the plan
-    accepts them (an even number of tile columns per frame)."""
+    """--qsort auto turns radius-sorted query groups on where the plan accepts
+    them (at most four tile rows per frame) and a tile-column strip holds more
+    than one tile."""
+    import dataclasses
     import pytest
     from sparse_attention_video_tra_b200 import TRA_FLAG_QSORT, TraError, synth
     W = synth.WORKLOADS
-    assert bench.query_group_flags("auto", W["wan720"]) == TRA_FLAG_QSORT       # 10 tile columns
+    assert bench.query_group_flags("auto", W["wan720"]) == TRA_FLAG_QSORT       # 3 tile rows of 16
     assert bench.query_group_flags("auto", W["hunyuan720"]) == TRA_FLAG_QSORT
     assert bench.query_group_flags("auto", W["len4x"]) == TRA_FLAG_QSORT
-    assert bench.query_group_flags("auto", W["wan480"]) == 0                    # 13 tile columns
+    assert bench.query_group_flags("auto", W["wan480"]) == 0                    # 1 tile row of 32
+    assert bench.query_group_flags("on", W["wan480"]) == TRA_FLAG_QSORT
     assert bench.query_group_flags("off", W["wan720"]) == 0
+    tall = dataclasses.replace(W["wan720"], H=200, W=200)                      # 13 tile rows
+    assert bench.query_group_flags("auto", tall) == 0
     with pytest.raises(TraError):
-        bench.query_group_flags("on", W["wan480"])
+        bench.query_group_flags("on", tall)

@@ -129,7 +129,7 @@ def test_wan720_full_size_qsort(run):
     r_nat[:, nat[nat >= 0]] = rad[sel].cpu().numpy()[:, nat >= 0]
     r_nat = r_nat.reshape(-1)
     perm, members = oracle.query_groups(r_nat, G, (T, H, W), (i.tile_h, i.tile_w))
-    np.testing.assert_array_equal(plan.group_view(mask)[sel].cpu().numpy(), perm)
+    np.testing.assert_array_equal(plan.group_view(mask)[sel].cpu().numpy().view(np.uint16), perm)
     Hg = gh.to_natural(run.H[sel], i).cpu().numpy().reshape(G * N)
     for t in rng.choice(i.n_tiles, size=3, replace=False):
         for gi, g in enumerate(sel):
@@ -149,4 +149,75 @@ def test_wan720_full_size_qsort(run):
     queries = np.sort(rng.choice(G * N, size=24, replace=False))
     Oref = oracle.attention(qb, kb, vb, r_nat, G, (T, H, W), d, wl.gamma, wl.Rt, queries=queries)
     gh.check_attention(o[queries], Oref)
+    plan.close()
+
+
+@pytest.mark.parametrize("metric", [oracle.CHEBYSHEV, oracle.DISK], ids=["square", "disk"])
+def test_wan720_every_cta_of_the_grouped_launch(run, metric):
+    """The benchmark's own configuration (TRA_FLAG_QSORT: radius-sorted
+    tile-column strips) at full size, covering every CTA of the attention
+    launch: each CTA takes slot s of frames 2f and 2f + 1 (frame 20 has no
+    partner), and one query of each of its two slots is checked against the
+    oracle -- radius bit-exact, output row within max-abs 1e-2 / mean-abs
+    1e-3 -- for two heads, with the Chebyshev square and with the disk.  The
+    group order equals the oracle's everywhere, and one group list per frame
+    pair equals the oracle's block mask of that group's members."""
+    wl, i = run.wl, run.info
+    T, H, W, d, N = wl.T, wl.H, wl.W, wl.d, wl.N
+    disk = metric == oracle.DISK
+    plan = _plan(run, tra.TRA_FLAG_QSORT | (tra.TRA_FLAG_DISK if disk else 0))
+    mask, out = plan.new_mask(), plan.new_out()
+    plan.radius_and_mask(run.H, mask)
+    plan.attention(run.q, run.k, run.v[0], mask, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    rng = np.random.default_rng(29 + metric)
+    sel = [0, wl.heads - 1]
+    G = len(sel)
+    tpf = i.n_tiles_h * i.n_tiles_w
+    nat = gh.tile_major_index(i)
+    rad, cnt, pairs, lst = plan.mask_views(mask)
+    r_nat = np.zeros((G, N), np.int32)
+    r_nat[:, nat[nat >= 0]] = rad[sel].cpu().numpy()[:, nat >= 0]
+    r_nat = r_nat.reshape(-1)
+    Hg = gh.to_natural(run.H[sel], i).cpu().numpy().reshape(G * N)
+    perm, members = oracle.query_groups(r_nat, G, (T, H, W), (i.tile_h, i.tile_w))
+    np.testing.assert_array_equal(plan.group_view(mask)[sel].cpu().numpy().view(np.uint16), perm)
+    # the launch: CTA p takes slot s = p % tpf of frames 2f and 2f + 1
+    slots = []
+    n_cta = (T + 1) // 2 * tpf
+    for p in range(n_cta):
+        qa = 2 * (p // tpf) * tpf + p % tpf
+        slots += [qa] + ([qa + tpf] if qa + tpf < i.n_tiles else [])
+    queries = []
+    for gi in range(G):
+        for a in slots:
+            m = members[gi * i.n_tiles + a]
+            queries.append(int(rng.choice(m[m >= 0])))
+    queries = np.array(sorted(set(queries)))
+    assert len(queries) >= 0.99 * G * i.n_tiles          # one query per slot of every CTA
+    r_ref, _, _ = oracle.radius(Hg[queries], G, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin,
+                                queries=queries, metric=metric)
+    np.testing.assert_array_equal(r_nat[queries], r_ref)
+    bits = lambda x: gh.bf16_bits(gh.to_natural(x[sel], i))     # noqa: E731
+    qb, kb, vb = bits(run.q), bits(run.k), bits(run.v[0])
+    o = gh.to_natural(out[sel], i).float().cpu().numpy().reshape(G * N, d)
+    Oref = oracle.attention(qb, kb, vb, r_nat, G, (T, H, W), d, wl.gamma, wl.Rt, queries=queries, metric=metric)
+    gh.check_attention(o[queries], Oref)
+    # one group list per frame pair and head
+    for f in range(0, T, 2):
+        a = f * tpf + int(rng.integers(tpf))
+        for gi, g in enumerate(sel):
+            mem = members[gi * i.n_tiles + a][None]
+            row = oracle.block_mask_sets(r_nat, G, (T, H, W), wl.gamma, wl.Rt, (i.tile_h, i.tile_w), mem,
+                                         metric=metric)[0]
+            n = int(cnt[g, a])
+            e = lst[g, a, :n].cpu().numpy().view(np.uint16).astype(np.int64)
+            dense = np.zeros(i.n_tiles, np.uint8)
+            dense[e & 0x7FFF] = np.where(e & 0x8000, 3, 1)
+            np.testing.assert_array_equal(dense, row)
+            q = mem[0][mem[0] >= 0]
+            _, c_mem, _ = oracle.radius(Hg[q], G, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, queries=q,
+                                        metric=metric)
+            assert int(pairs[g, a]) == int(c_mem.sum())
     plan.close()

@@ -92,6 +92,31 @@ def test_list_entry_beyond_its_own_tiles_reach_is_reported():
     assert plan.status() == 0
 
 
+def test_group_entry_past_the_strip_is_reported():
+    """With radius-sorted groups each slot names a strip row; a row past the
+    strip (128 * n_tiles_h or more) is recorded, never followed."""
+    T, H, W, G, d, gamma, Rt, Bmin = C
+    plan = tra.Plan(T, H, W, G, d, 1.0, 0.5, gamma, Rt, Bmin, tra.TRA_FLAG_QSORT | tra.tra_flag_tile_w(8))
+    i = plan.info
+    q, k, v = synth.make_qkv(T, H, W, G, d, 5, device="cuda", dtype=torch.bfloat16)
+    qt, kt, vt = (gh.to_tile_major(x, i) for x in (q, k, v))
+    Ht = torch.empty(G, i.N_pad, device="cuda")
+    plan.entropy(qt, kt, Ht)
+    mask = plan.new_mask()
+    plan.radius_and_mask(Ht, mask)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    bad = mask.clone()
+    plan.group_view(bad)[1, 2, 5] = 0x7FFF
+    out = plan.new_out()
+    plan.attention(qt, kt, vt, bad, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 6
+    plan.attention(qt, kt, vt, mask, out)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+
+
 def test_results_are_bit_identical_across_runs():
     plan, (qt, kt, vt), Ht, mask = _setup(seed=9)
     i = plan.info

@@ -5,11 +5,11 @@ and for the block mask of explicit query sets.
 * Block masks of sets equal the tile block mask when the sets are the tiles
   (two independent oracle paths), and a dense numpy brute force for arbitrary
   sets (bruteforce.token_mask).
-* The two groups of a pair partition its 256 rows, every radius of the first
-  group is at most every radius of the second, equal radii keep row order,
-  and pad rows come first.
-* Token voting is an OR, so the union of the two groups' active tiles equals
-  the union of the pair's two tiles' active tiles."""
+* The groups of a strip (one tile column of one frame) partition its
+  128*nTh rows, radii never decrease from one group to the next or inside a
+  group, equal radii keep row order, and pad rows come first.
+* Token voting is an OR, so the union of a strip's groups' active tiles
+  equals the union of the strip's tiles' active tiles."""
 import numpy as np
 import pytest
 
@@ -78,37 +78,50 @@ def test_sets_equal_bruteforce(disk):
     assert n_full > 0
 
 
-def test_groups_partition_pairs_sorted_by_radius():
-    T, H, W, G = 3, 20, 16, 2
-    tile = (16, 8)
+def _strip_tiles(grid, tile):
+    T, H, W = grid
+    th, tw = tile
+    nTh, nTw = -(-H // th), -(-W // tw)
+    return [[t * nTh * nTw + u * nTw + c for u in range(nTh)] for t in range(T) for c in range(nTw)]
+
+
+@pytest.mark.parametrize("grid,tile", [((3, 20, 16), (16, 8)), ((2, 45, 80), (16, 8)), ((2, 30, 20), (8, 16)),
+                                       ((3, 8, 12), (32, 4))])
+def test_groups_partition_strips_sorted_by_radius(grid, tile):
+    T, H, W = grid
+    G = 2
     N = T * H * W
     r = np.random.default_rng(3).integers(0, 9, G * N).astype(np.int32)
-    perm, mem = oracle.query_groups(r, G, (T, H, W), tile)
+    perm, mem = oracle.query_groups(r, G, grid, tile)
     nQ = perm.shape[1]
-    tm = _tile_members(G, (T, H, W), tile)
+    tm = _tile_members(G, grid, tile)
     for g in range(G):
-        for a in range(0, nQ, 2):
-            both = np.concatenate([perm[g, a], perm[g, a + 1]]).astype(np.int64)
-            assert sorted(both.tolist()) == list(range(256))
-            pair_rows = np.concatenate([tm[g * nQ + a], tm[g * nQ + a + 1]])
-            rad = np.where(pair_rows >= 0, r[np.maximum(pair_rows, 0)], -1)
-            ordered = rad[both]
+        for tiles in _strip_tiles(grid, tile):
+            U = len(tiles)
+            allp = np.concatenate([perm[g, a] for a in tiles]).astype(np.int64)
+            assert sorted(allp.tolist()) == list(range(128 * U))
+            strip_rows = np.concatenate([tm[g * nQ + a] for a in tiles])
+            rad = np.where(strip_rows >= 0, r[np.maximum(strip_rows, 0)], -1)
+            ordered = rad[allp]
             assert np.all(np.diff(ordered) >= 0)                     # sorted by radius (pads, -1, first)
             for v in np.unique(ordered):
-                rows = both[ordered == v]
+                rows = allp[ordered == v]
                 assert np.all(np.diff(rows) > 0)                     # ties keep row order
-            for k in range(2):
-                np.testing.assert_array_equal(mem[g * nQ + a + k], pair_rows[perm[g, a + k].astype(np.int64)])
+            for u, a in enumerate(tiles):
+                np.testing.assert_array_equal(mem[g * nQ + a], strip_rows[perm[g, a].astype(np.int64)])
 
 
-def test_group_union_equals_tile_union():
-    T, H, W, G = 3, 20, 16, 2
-    tile = (16, 8)
+@pytest.mark.parametrize("grid,tile", [((3, 20, 16), (16, 8)), ((2, 30, 20), (8, 16))])
+def test_group_union_equals_tile_union(grid, tile):
+    T, H, W = grid
+    G = 2
     N = T * H * W
     r = np.random.default_rng(4).integers(0, 9, G * N).astype(np.int32)
-    _, mem = oracle.query_groups(r, G, (T, H, W), tile)
-    grp = oracle.block_mask_sets(r, G, (T, H, W), 0.8, 2, tile, mem) > 0
-    til = oracle.block_mask(r, G, (T, H, W), 0.8, 2, tile, tile) > 0
-    np.testing.assert_array_equal(grp[0::2] | grp[1::2], til[0::2] | til[1::2])
-    # and sorting never adds work: the groups list at most as many tiles as the tiles do
-    assert grp.sum() <= til.sum()
+    _, mem = oracle.query_groups(r, G, grid, tile)
+    grp = oracle.block_mask_sets(r, G, grid, 0.8, 2, tile, mem) > 0
+    til = oracle.block_mask(r, G, grid, 0.8, 2, tile, tile) > 0
+    nQ = grp.shape[0] // G
+    for g in range(G):
+        for tiles in _strip_tiles(grid, tile):
+            rows = [g * nQ + a for a in tiles]
+            np.testing.assert_array_equal(np.any(grp[rows], axis=0), np.any(til[rows], axis=0))
