@@ -259,20 +259,19 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // 16 bytes per load; rows outside the grid are zeros
         constexpr int CH = D / 8;                           // 16-byte chunks of a row
         const int np = hasB ? 2 : 1;
-        int tqs[2], tcs[2];
-        for (int sl = 0; sl < 2; ++sl) {
-            int trx;
-            tile_coords(G, sl ? (hasB ? qb : qa) : qa, tqs[sl], trx, tcs[sl]);
-        }
+        int tqa_, tra_, tca_, tqb_, trb_, tcb_;
+        tile_coords(G, qa, tqa_, tra_, tca_);
+        tile_coords(G, hasB ? qb : qa, tqb_, trb_, tcb_);
         for (int e = tid; e < 128 * np * CH; e += C::THREADS) {
             const int d = e / CH, ch = e - d * CH;
             const int sl = d >> 7, dr = d & 127;
             const int l = (sl ? grp_b : grp_a)[dr];
-            const int hq = (l >> 7) * G.th + ((l & 127) >> TWL), wq = tcs[sl] * TW + (l & (TW - 1));
+            const int tq = sl ? tqb_ : tqa_, tcq = sl ? tcb_ : tca_;
+            const int hq = (l >> 7) * G.th + ((l & 127) >> TWL), wq = tcq * TW + (l & (TW - 1));
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
             if (hq < G.H && wq < G.W) {
-                const int tl = (tqs[sl] * G.nTh + (l >> 7)) * G.nTw + tcs[sl];
-                const size_t qrow = io_row(G, g, tqs[sl], hq, wq, tl * 128 + (l & 127));
+                const int tl = (tq * G.nTh + (l >> 7)) * G.nTw + tcq;
+                const size_t qrow = io_row(G, g, tq, hq, wq, tl * 128 + (l & 127));
                 val = __ldg(reinterpret_cast<const uint4*>(qraw) + qrow * CH + ch);
             }
             const int pn = ch >> 3, cc = ch & 7;
@@ -390,8 +389,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     issue_unlock(s_lock);
                 }
                 if (!release_v()) { ok = false; break; }
-                if (!role_wait(&p_full[w], cnt & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                // V has usually landed long before the softmax ends: wait for it
+                // first, so that only the lock follows the softmax's hand-off
                 if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
+                if (!role_wait(&p_full[w], cnt & 1, G.wait_ns, s_abort)) { ok = false; break; }
                 if (!issue_lock(s_lock, G.wait_ns, s_abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll

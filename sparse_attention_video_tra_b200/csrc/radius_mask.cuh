@@ -46,37 +46,60 @@ __device__ __forceinline__ int hw_at(const Geom& G, const uint16_t* tab, int r, 
     return tab ? (int)tab[dl * (G.r_cap + 1) + r] : halfwidth(r, G.g[dl]);
 }
 
-// clipped neighbourhood count c(r) of the query at (t, h, w): per frame the
-// Chebyshev square is a clipped rectangle; the disk sums, key row by key row,
-// the clipped width 2*isqrt(s^2 - dh^2) + 1
-template <bool DISK>
-__device__ __forceinline__ long long nbr_count(const Geom& G, const uint16_t* tab, int t, int h, int w, int r)
+// Per query: what the neighbourhood count needs besides r.  Frames t + dt
+// and t - dt hold the same clipped rectangle, so the count is
+//   c(r) = P(0) + 2 * sum_{1 <= dt <= lo} P(dt) + sum_{lo < dt <= hi} P(dt)
+// with lo / hi the smaller / larger of the reaches min(Rt', T-1-t) and
+// min(Rt', t) on the two sides, and P(dt) the in-frame count at half-width
+// s(r, dt).
+struct CountCtx {
+    int h, w, hb, wb;      // distances to the top / left and bottom / right edges
+    int lo, hi;            // both sides within lo frames; one side up to hi
+};
+
+__device__ __forceinline__ CountCtx count_ctx(const Geom& G, int t, int h, int w)
 {
-    long long c = 0;
-    for (int dl = 0; dl <= G.rte; ++dl) {
-        const int m = (t + dl < G.T ? 1 : 0) + (dl > 0 && t - dl >= 0 ? 1 : 0);
-        if (m == 0) break;                         // farther frames are out of the grid too
-        const int s = hw_at(G, tab, r, dl);
-        if constexpr (DISK) {
-            // key rows h - k (k <= up) and h + k (k <= dn) share the half-width
-            // isqrt(s^2 - k^2)
-            const int sc = min(s, TRA_DISK_S_CLAMP);
-            const int up = min(sc, h), dn = min(sc, G.H - 1 - h);
-            const int kmax = max(up, dn), s2 = sc * sc;
-            long long X = 0;
-            for (int k = 0; k <= kmax; ++k) {
-                const int half = isqrt_floor(s2 - k * k);
-                const int wid = min(G.W - 1, w + half) - max(0, w - half) + 1;
-                X += k == 0 ? wid : (k <= up ? wid : 0) + (k <= dn ? wid : 0);
-            }
-            c += m * X;
-        } else {
-            const int X = min(h, s) + min(G.H - 1 - h, s) + 1;
-            const int Y = min(w, s) + min(G.W - 1 - w, s) + 1;
-            c += (long long)(m * X) * Y;
+    CountCtx x;
+    x.h = h; x.w = w;
+    x.hb = G.H - 1 - h; x.wb = G.W - 1 - w;
+    const int fwd = min(G.rte, G.T - 1 - t), bwd = min(G.rte, t);
+    x.lo = min(fwd, bwd);
+    x.hi = max(fwd, bwd);
+    return x;
+}
+
+// in-frame clipped count at half-width s: the Chebyshev square is a clipped
+// rectangle; the disk sums, key row by key row, the clipped width
+// 2*isqrt(s^2 - dh^2) + 1
+template <bool DISK>
+__device__ __forceinline__ int frame_count(const Geom& G, const CountCtx& x, int s)
+{
+    if constexpr (DISK) {
+        // key rows h - k (k <= up) and h + k (k <= dn) share the half-width
+        // isqrt(s^2 - k^2)
+        const int sc = min(s, TRA_DISK_S_CLAMP);
+        const int up = min(sc, x.h), dn = min(sc, x.hb);
+        const int kmax = max(up, dn), s2 = sc * sc;
+        int X = 0;
+        for (int k = 0; k <= kmax; ++k) {
+            const int half = isqrt_floor(s2 - k * k);
+            const int wid = min(x.wb, half) + min(x.w, half) + 1;
+            X += k == 0 ? wid : (k <= up ? wid : 0) + (k <= dn ? wid : 0);
         }
+        return X;
+    } else {
+        return (min(x.h, s) + min(x.hb, s) + 1) * (min(x.w, s) + min(x.wb, s) + 1);
     }
-    return c;
+}
+
+// clipped neighbourhood count c(r) (at most N < 2^31)
+template <bool DISK>
+__device__ __forceinline__ long long nbr_count(const Geom& G, const uint16_t* tab, const CountCtx& x, int r)
+{
+    int one = 0, two = 0;
+    for (int dl = 1; dl <= x.lo; ++dl) two += frame_count<DISK>(G, x, hw_at(G, tab, r, dl));
+    for (int dl = x.lo + 1; dl <= x.hi; ++dl) one += frame_count<DISK>(G, x, hw_at(G, tab, r, dl));
+    return (long long)frame_count<DISK>(G, x, hw_at(G, tab, r, 0)) + 2ll * two + one;
 }
 
 // Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))): a*H and + b rounded
@@ -93,6 +116,7 @@ template <bool DISK>
 __device__ __forceinline__ int find_radius(const Geom& G, const uint16_t* tab, int t, int h, int w, long long bh,
                                            long long& c)
 {
+    const CountCtx x = count_ctx(G, t, h, w);
     int lo = 0, hi = G.r_cap;
     if constexpr (DISK) {
         // the disk lies inside the square of the same half-width, so its
@@ -100,17 +124,19 @@ __device__ __forceinline__ int find_radius(const Geom& G, const uint16_t* tab, i
         // that bracket reaches the budget, else the rest up to r_cap
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (nbr_count<false>(G, tab, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+            if (nbr_count<false>(G, tab, x, mid) >= bh) hi = mid; else lo = mid + 1;
         }
         const int r2 = min(G.r_cap, 2 * lo + 2);
-        if (nbr_count<true>(G, tab, t, h, w, r2) >= bh) hi = r2;
+        if (nbr_count<true>(G, tab, x, r2) >= bh) hi = r2;
         else { lo = min(r2 + 1, G.r_cap); hi = G.r_cap; }
     }
+    long long c_hi = -1;                  // the count at hi, once evaluated
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (nbr_count<DISK>(G, tab, t, h, w, mid) >= bh) hi = mid; else lo = mid + 1;
+        const long long cm = nbr_count<DISK>(G, tab, x, mid);
+        if (cm >= bh) { hi = mid; c_hi = cm; } else lo = mid + 1;
     }
-    c = nbr_count<DISK>(G, tab, t, h, w, lo);
+    c = c_hi >= 0 ? c_hi : nbr_count<DISK>(G, tab, x, lo);
     return lo;
 }
 
@@ -131,8 +157,10 @@ __host__ __device__ inline int mask_smem_bytes(int rte, int nTh, int r_cap, bool
     return mask_tab_bytes(rte, r_cap, tab) + U * (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
 }
 
-template <bool DISK, bool QS>
-__global__ void __launch_bounds__(MASK_MAX_ROWS) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
+// MAXT: the block size the instance is built for (128 * U); the register
+// budget follows from it (three strips of three tiles per SM, or eight tiles)
+template <bool DISK, bool QS, int MAXT>
+__global__ void __launch_bounds__(MAXT, MAXT == 128 ? 8 : (MAXT == 384 ? 3 : 2)) radius_mask_kernel(const Geom G, const float* __restrict__ Hent,
                                                                     uint8_t* __restrict__ mask)
 {
     extern __shared__ __align__(16) uint8_t mask_dyn[];
@@ -165,12 +193,10 @@ __global__ void __launch_bounds__(MASK_MAX_ROWS) radius_mask_kernel(const Geom G
     auto strip_tile = [&](int uu) { return (t * G.nTh + tr0 + uu) * G.nTw + tc; };
 
     if (tab) {
-        const int n = (G.rte + 1) * (G.r_cap + 1);
         uint16_t* wtab = reinterpret_cast<uint16_t*>(mask_dyn);
-        for (int e = tid; e < n; e += blockDim.x) {
-            const int dl = e / (G.r_cap + 1);
-            wtab[e] = (uint16_t)halfwidth(e - dl * (G.r_cap + 1), G.g[dl]);
-        }
+        for (int dl = 0; dl <= G.rte; ++dl)
+            for (int rr = tid; rr <= G.r_cap; rr += blockDim.x)
+                wtab[dl * (G.r_cap + 1) + rr] = (uint16_t)halfwidth(rr, G.g[dl]);
     }
     int* s_lo = grp_base + u * GS;                                // [rte + 1][nTh]
     int* s_hi = s_lo + (G.rte + 1) * RS;                          // [rte + 1][nTh]
@@ -209,11 +235,13 @@ __global__ void __launch_bounds__(MASK_MAX_ROWS) radius_mask_kernel(const Geom G
             }
         s_key[tid] = key;
         __syncthreads();
+        // keys of every other warp below `key` (independent searches, unrolled)
         int rank = lane;
-        for (int ow = 0; ow < 4 * U; ++ow) {
-            if (ow == warp) continue;
+#pragma unroll
+        for (int ow = 0; ow < MASK_MAX_ROWS / 32; ++ow) {
+            if (ow >= 4 * U || ow == warp) continue;
             const int* sk = s_key + ow * 32;
-            int lo = 0;                                           // keys of warp ow below `key`
+            int lo = 0;
 #pragma unroll
             for (int step = 16; step > 0; step >>= 1)
                 if (sk[lo + step - 1] < key) lo += step;
@@ -265,9 +293,8 @@ __global__ void __launch_bounds__(MASK_MAX_ROWS) radius_mask_kernel(const Geom G
             atomicMax(&s_full[u][dl][0], frl); atomicMin(&s_full[u][dl][1], frh);
             atomicMax(&s_full[u][dl][2], fcl); atomicMin(&s_full[u][dl][3], fch);
         }
-        const int r_lo = __reduce_min_sync(0xffffffffu, rl);
-        const int r_hi = __reduce_max_sync(0xffffffffu, rh);
-        for (int tr = r_lo; tr <= r_hi; ++tr) {
+        // the union of the members' column intervals over key tile row tr
+        auto row_union = [&](int tr) {
             const bool in = rl <= tr && tr <= rh;
             int c_lo = cl, c_hi = ch;
             if (DISK && in) {
@@ -285,6 +312,18 @@ __global__ void __launch_bounds__(MASK_MAX_ROWS) radius_mask_kernel(const Geom G
                 atomicMin(&s_lo[dl * RS + tr], lo);
                 atomicMax(&s_hi[dl * RS + tr], hi);
             }
+        };
+        if constexpr (QS) {
+            // a strip has at most TRA_MAX_STRIP_TILES tile rows: all of them,
+            // as independent reductions
+#pragma unroll
+            for (int tr = 0; tr < TRA_MAX_STRIP_TILES; ++tr)
+                if (tr < G.nTh) row_union(tr);
+        } else {
+            // a lone tile walks the warp's row range
+            const int r_lo = __reduce_min_sync(0xffffffffu, rl);
+            const int r_hi = __reduce_max_sync(0xffffffffu, rh);
+            for (int tr = r_lo; tr <= r_hi; ++tr) row_union(tr);
         }
     }
     __syncthreads();

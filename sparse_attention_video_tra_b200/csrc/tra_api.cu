@@ -196,8 +196,9 @@ extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void
         return true;
     };
     bool ok;
-    if (G.qsort) ok = G.disk ? go(tra::radius_mask_kernel<true, true>) : go(tra::radius_mask_kernel<false, true>);
-    else ok = G.disk ? go(tra::radius_mask_kernel<true, false>) : go(tra::radius_mask_kernel<false, false>);
+    if (!G.qsort) ok = G.disk ? go(tra::radius_mask_kernel<true, false, 128>) : go(tra::radius_mask_kernel<false, false, 128>);
+    else if (U <= 3) ok = G.disk ? go(tra::radius_mask_kernel<true, true, 384>) : go(tra::radius_mask_kernel<false, true, 384>);
+    else ok = G.disk ? go(tra::radius_mask_kernel<true, true, 512>) : go(tra::radius_mask_kernel<false, true, 512>);
     if (!ok) return TRA_ERR_CUDA;
     return launch_status();
 }
