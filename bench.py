@@ -584,12 +584,18 @@ def run_e2e(run, wl, calls, args, world):
     kernels read frame-major tensors through 4-D TMA boxes, no permute pass),
     and each call's output back to pinned host memory.
 
-    Heads are independent problems, so the heads are split into chunks, each
-    with its own plan and mask buffer: the first chunk's entropy starts once
-    its own Q and K are up, and only the last chunk's output of the last call
-    is copied after the compute ends.  Copies run on their own streams: V of
-    call c+1 goes up while call c computes, and each chunk's output comes down
-    while the next chunk computes (V and outputs are double buffered)."""
+    Copies run on their own streams and overlap compute, within a step and
+    across steps: Q and K are double-buffered by step, so the next step's
+    upload runs during this step's last attention calls; V and the outputs are
+    double-buffered by call, so V of call c+1 goes up while call c runs and
+    each output comes down while later work runs.  The fences (an event per
+    buffer) carry over from one step to the next; the timed region ends when
+    the last output has landed in host memory.
+
+    Heads are independent problems, so they may be split into chunks
+    (--e2e-chunks), each with its own plan and mask buffer; with the
+    cross-step overlap one chunk (one launch per call, no extra wave tails)
+    is the default."""
     from sparse_attention_video_tra_b200 import Plan, TRA_FLAG_NATURAL
     from sparse_attention_video_tra_b200.runner import shard_heads
     i = run.info
@@ -607,9 +613,9 @@ def run_e2e(run, wl, calls, args, world):
     run.plan.permute(run.k, tmp, False); hk.copy_(tmp)
     run.plan.permute(run.v[0], tmp, False); hv.copy_(tmp)
     del tmp
-    dq = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
-    dk = torch.empty_like(dq)
-    dv = [torch.empty_like(dq), torch.empty_like(dq)]
+    dq = [torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    dk = [torch.empty_like(dq[0]) for _ in range(2)]
+    dv = [torch.empty_like(dq[0]) for _ in range(2)]
     do = [torch.empty(shape, dtype=plans[0].out_dtype, device="cuda") for _ in range(2)]
     dH = torch.empty((i.heads, i.N), dtype=torch.float32, device="cuda")
     dmask = [p.new_mask() for p in plans]
@@ -617,42 +623,47 @@ def run_e2e(run, wl, calls, args, world):
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()                       # noqa: E731
+    # fences carried across steps (None: the buffer is free)
+    st = {"qk_free": [None, None], "v_free": [None, None], "o_free": [[None] * n_chunks for _ in range(2)],
+          "last": None, "n": 0}
 
     def step():
-        start = ev(); start.record(comp)
-        s_in.wait_event(start)
+        p = st["n"] & 1
+        st["n"] += 1
+        if st["qk_free"][p] is not None:                   # the step two back no longer reads set p
+            s_in.wait_event(st["qk_free"][p])
         qk_in = []
         with torch.cuda.stream(s_in):
             for h in sl:
-                dq[h].copy_(hq[h], non_blocking=True)
-                dk[h].copy_(hk[h], non_blocking=True)
+                dq[p][h].copy_(hq[h], non_blocking=True)
+                dk[p][h].copy_(hk[h], non_blocking=True)
                 qk_in.append(ev()); qk_in[-1].record(s_in)
-        for p, h, m, e in zip(plans, sl, dmask, qk_in):
+        for pl, h, m, e in zip(plans, sl, dmask, qk_in):
             comp.wait_event(e)
-            p.entropy(dq[h], dk[h], dH[h], wl.key_stride, stream=comp)
-            p.radius_and_mask(dH[h], m, stream=comp)
-        v_free = [start, start]                            # buffer b may be refilled
-        o_free = [[start] * n_chunks for _ in range(2)]    # chunk of buffer b may be rewritten
-        last = start
+            pl.entropy(dq[p][h], dk[p][h], dH[h], wl.key_stride, stream=comp)
+            pl.radius_and_mask(dH[h], m, stream=comp)
+        done = None
         for c in range(calls):
             b = c & 1
-            s_in.wait_event(v_free[b])
+            if st["v_free"][b] is not None:
+                s_in.wait_event(st["v_free"][b])
             with torch.cuda.stream(s_in):
                 dv[b].copy_(hv, non_blocking=True)
                 v_in = ev(); v_in.record(s_in)
             comp.wait_event(v_in)
-            for q, (p, h, m) in enumerate(zip(plans, sl, dmask)):
-                comp.wait_event(o_free[b][q])
-                p.attention(dq[h], dk[h], dv[b][h], m, do[b][h], stream=comp)
+            for q, (pl, h, m) in enumerate(zip(plans, sl, dmask)):
+                if st["o_free"][b][q] is not None:
+                    comp.wait_event(st["o_free"][b][q])
+                pl.attention(dq[p][h], dk[p][h], dv[b][h], m, do[b][h], stream=comp)
                 done = ev(); done.record(comp)
                 s_out.wait_event(done)
                 with torch.cuda.stream(s_out):
                     ho[h].copy_(do[b][h], non_blocking=True)
                     out_done = ev(); out_done.record(s_out)
-                o_free[b][q] = out_done
-                last = out_done
-            v_free[b] = done
-        comp.wait_event(last)
+                st["o_free"][b][q] = out_done
+                st["last"] = out_done
+            st["v_free"][b] = done
+        st["qk_free"][p] = done
 
     for _ in range(args.warmup):
         step()
@@ -662,6 +673,7 @@ def run_e2e(run, wl, calls, args, world):
     e0.record(comp)
     for _ in range(args.steps):
         step()
+    comp.wait_event(st["last"])                            # every output in host memory
     e1.record(comp)
     torch.cuda.synchronize()
     barrier(world)
@@ -676,7 +688,8 @@ def run_e2e(run, wl, calls, args, world):
     return {"value": round(val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": nbytes * (2 + calls),
             "d2h_bytes_per_step": obytes * calls, "ms_per_step": round(secs * 1000.0 / args.steps, 3),
             "head_chunks": n_chunks,
-            "layout": "natural [heads][T][H][W][d]; heads in chunks, copies overlapped with compute on two copy streams"}
+            "layout": "natural [heads][T][H][W][d]; copies on two copy streams, overlapped with compute "
+                      "within and across steps (Q/K double-buffered by step, V and outputs by call)"}
 
 
 def main(argv=None):
@@ -698,8 +711,8 @@ def main(argv=None):
                     help="radius-sorted query groups (TRA_FLAG_QSORT): auto = when the frame has an even "
                          "number of tile columns")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=4,
-                    help="head chunks of the end-to-end leg (each its own plan; copies overlap the other chunks)")
+    ap.add_argument("--e2e-chunks", type=int, default=1,
+                    help="head chunks of the end-to-end leg (each its own plan and launches)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     raw = list(sys.argv[1:] if argv is None else argv)
