@@ -201,12 +201,17 @@ entropy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float c = G.scale_log2;
         float m = -1e30f, Z = 0.f, A = 0.f;
         bool ok = w == 0 || hasB;
+        // (tile row, tile column) of key tile j*stride, advanced by the stride
+        // (sr, sc) = stride mod tiles-per-frame, so the loop divides nothing
+        const int smod = stride % G.tiles_per_frame, sr = smod / G.nTw, sc = smod - sr * G.nTw;
+        int trk = 0, tck = 0;
         for (int j = 0; ok && j < n; ++j) {
-            const int kb = j * stride;
-            int tk, trk, tck;
-            tile_coords(G, kb, tk, trk, tck);
             const int khv = min(G.th, G.H - trk * G.th), kwv = min(TW, G.W - tck * TW);
             const bool edge = khv < G.th || kwv < TW;
+            tck += sc;
+            trk += sr;
+            if (tck >= G.nTw) { tck -= G.nTw; ++trk; }
+            if (trk >= G.nTh) trk -= G.nTh;
             const int bs = w * 2 + (j & 1);
             const bool got = role_wait(&s_full[bs], (j >> 1) & 1, G.wait_ns, s_abort);
             if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
