@@ -143,10 +143,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // the CTA's two query tiles, or with radius-sorted groups two mask slots of
     // like size and heavily overlapping lists: slot s of frames 2f and 2f + 1
     // (both small-radius groups or both large-radius ones, one frame apart),
-    // so that the two per-slot chains stay about equally long and interleave
+    // so that the two per-slot chains stay about equally long and interleave.
+    // An odd last frame has no partner frame: its slots pair with each other
+    // (slots 2k and 2k + 1 of that frame, neighbouring strips), so that no
+    // CTA runs a lone chain while a slot of the frame is left to pair with.
     const int tpf = G.tiles_per_frame;
-    const int qa = G.qsort ? 2 * (pair / tpf) * tpf + pair % tpf : 2 * pair;
-    const int qb = G.qsort ? qa + tpf : qa + 1;
+    const int paired = (G.T / 2) * tpf;                 // CTAs of the frame pairs
+    int qa = 2 * pair, qb = qa + 1;
+    if (G.qsort && pair < paired) {
+        qa = 2 * (pair / tpf) * tpf + pair % tpf;
+        qb = qa + tpf;
+    } else if (G.qsort) {
+        qa = (G.T - 1) * tpf + 2 * (pair - paired);
+        qb = qa + 1;
+    }
     const bool hasB = qb < G.nQ;
     const int32_t* counts = reinterpret_cast<const int32_t*>(mask + G.off_count) + (size_t)g * G.nQ;
     const uint16_t* lists = reinterpret_cast<const uint16_t*>(mask + G.off_list) + (size_t)g * G.nQ * G.list_cap;

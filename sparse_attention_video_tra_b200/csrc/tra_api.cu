@@ -99,8 +99,9 @@ tra_status run_attention(const tra::Geom& G, const CUtensorMap& q, const CUtenso
     if (smem > kMaxSmem) return TRA_ERR_UNSUPPORTED;
     if (!set_smem(kern, smem)) return TRA_ERR_CUDA;
     // two query tiles per CTA; with radius-sorted groups, the same slot of
-    // frames 2f and 2f + 1
-    const int ctas = G.qsort ? (G.T + 1) / 2 * G.tiles_per_frame : (G.nQ + 1) / 2;
+    // frames 2f and 2f + 1, then an odd last frame's slots two by two
+    const int ctas = G.qsort ? G.T / 2 * G.tiles_per_frame + (G.T % 2) * ((G.tiles_per_frame + 1) / 2)
+                             : (G.nQ + 1) / 2;
     kern<<<dim3(ctas, G.G), C::THREADS, smem, st>>>(q, k, v, G, mask, out, qraw);
     return launch_status();
 }

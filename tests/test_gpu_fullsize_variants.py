@@ -156,8 +156,8 @@ def test_wan720_full_size_qsort(run):
 def test_wan720_every_cta_of_the_grouped_launch(run, metric):
     """The benchmark's own configuration (TRA_FLAG_QSORT: radius-sorted
     tile-column strips) at full size, covering every CTA of the attention
-    launch: each CTA takes slot s of frames 2f and 2f + 1 (frame 20 has no
-    partner), and one query of each of its two slots is checked against the
+    launch: each CTA takes slot s of frames 2f and 2f + 1, or two adjacent
+    slots of the odd last frame 20, and one query of each of its slots is checked against the
     oracle -- radius bit-exact, output row within max-abs 1e-2 / mean-abs
     1e-3 -- for two heads, with the Chebyshev square and with the disk.  The
     group order equals the oracle's everywhere, and one group list per frame
@@ -183,12 +183,20 @@ def test_wan720_every_cta_of_the_grouped_launch(run, metric):
     Hg = gh.to_natural(run.H[sel], i).cpu().numpy().reshape(G * N)
     perm, members = oracle.query_groups(r_nat, G, (T, H, W), (i.tile_h, i.tile_w))
     np.testing.assert_array_equal(plan.group_view(mask)[sel].cpu().numpy().view(np.uint16), perm)
-    # the launch: CTA p takes slot s = p % tpf of frames 2f and 2f + 1
+    # the launch: CTA p < (T // 2) * tpf takes slot s = p % tpf of frames 2f
+    # and 2f + 1; the rest take slots 2k, 2k + 1 of the odd last frame
     slots = []
-    n_cta = (T + 1) // 2 * tpf
+    paired = T // 2 * tpf
+    n_cta = paired + (T % 2) * ((tpf + 1) // 2)
     for p in range(n_cta):
-        qa = 2 * (p // tpf) * tpf + p % tpf
-        slots += [qa] + ([qa + tpf] if qa + tpf < i.n_tiles else [])
+        if p < paired:
+            qa = 2 * (p // tpf) * tpf + p % tpf
+            qb = qa + tpf
+        else:
+            qa = (T - 1) * tpf + 2 * (p - paired)
+            qb = qa + 1
+        slots += [qa] + ([qb] if qb < i.n_tiles else [])
+    assert sorted(slots) == list(range(i.n_tiles))         # every slot in exactly one CTA
     queries = []
     for gi in range(G):
         for a in slots:

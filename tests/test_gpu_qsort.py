@@ -39,6 +39,7 @@ CASES = [
     (3, 9, 60, 1, 128, 0.9, 2, 3, 32),      # (1,4,32) tiles
     (2, 45, 80, 1, 128, 0.8, 1, 8, 0),      # 720p frame, (1,16,8) tiles
     (3, 30, 20, 2, 64, 0.8, 2, 8, 16),      # (1,8,16) tiles: four tile rows, odd tile columns
+    (3, 48, 24, 2, 64, 0.8, 2, 8, 8),       # (1,16,8) tiles, 3x3 per frame: the odd last frame's slots pair up, one is left alone
 ]
 
 
