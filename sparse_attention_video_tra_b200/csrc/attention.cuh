@@ -399,6 +399,15 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     issue_unlock(s_lock);
                 }
                 if (!release_v()) { ok = false; break; }
+                // This tile's next listed entry j' joins this group when its K has
+                // landed: the tensor pipe runs the MMAs of one thread in order, so
+                // the QK overwrites S (holding P) only after this PV has read it.
+                // Only j' <= j + KST is looked at: every earlier entry of j''s
+                // ring stage has then been waited for by this thread, so the
+                // parity test names j''s own landing.
+                int jn = j + 1;
+                while (jn < n && jn <= j + C::KST && !(merged[jn] & in_bit)) ++jn;
+                const bool has_next = jn < n && jn <= j + C::KST;
                 // V has usually landed long before the softmax ends: wait for it
                 // first, so that only the lock follows the softmax's hand-off
                 if (!role_wait(&v_full[vs], (j / C::VST) & 1, G.wait_ns, s_abort)) { ok = false; break; }
@@ -410,21 +419,15 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_ts(tmem + col_o(w), tmem + col_s(w) + kk * 8,
                            smem_desc_sw128(sVa + vs * C::TILE + kk * 2048, C::PANEL, 1024), IDESC_PV,
                            (cnt > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&pv_done[w]);
                 mma_commit(&v_empty[vs]);
-                // This tile's next listed entry j' joins this group when its K has
-                // landed: the tensor pipe runs the MMAs of one thread in order, so
-                // the QK overwrites S (holding P) only after this PV has read it.
-                // Only j' <= j + KST is looked at: every earlier entry of j''s
-                // ring stage has then been waited for by this thread, so the
-                // parity test names j''s own landing.
-                int jn = j + 1;
-                while (jn < n && jn <= j + C::KST && !(merged[jn] & in_bit)) ++jn;
-                if (jn < n && jn <= j + C::KST && mbar_test(&k_full[jn % C::KST], (jn / C::KST) & 1)) {
+                if (has_next && mbar_test(&k_full[jn % C::KST], (jn / C::KST) & 1)) {
                     tc_fence_after();
                     issue_qk(jn);
                     qk_ahead = jn;
                 }
+                // only the epilogue waits for the last PV; a commit covers every
+                // earlier MMA of this thread, so this one may follow the QK
+                mma_commit(&pv_done[w]);
                 issue_unlock(s_lock);
                 ++cnt;
             }
