@@ -310,6 +310,44 @@ def test_bounded_wait_gives_up_and_context_survives():
     assert torch.isfinite(gh.to_natural(out, i).float()).all()
 
 
+@pytest.mark.parametrize("extra", [tra.TRA_FLAG_QSORT, tra.TRA_FLAG_NATURAL, tra.TRA_FLAG_QSORT | tra.TRA_FLAG_DISK],
+                         ids=["groups", "natural", "groups-disk"])
+def test_bounded_wait_other_paths(extra):
+    """The same give-up hook on the other code paths: radius-sorted groups (Q
+    gathered before the roles start, no Q barrier), the natural layout (4-D
+    TMA boxes), the disk, and the calibration kernel.  Each records a timeout
+    and returns; a normal call afterwards works and reports OK."""
+    T, H, W, G, d = 5, 17, 23, 2, 128
+    flags = extra | tra.tra_flag_tile_w(8)
+    good = tra.Plan(T, H, W, G, d, 1.0, math.log(0.3), 0.8, 3, 8, flags)
+    bad = tra.Plan(T, H, W, G, d, 1.0, math.log(0.3), 0.8, 3, 8, flags | tra.TRA_FLAG_DEBUG_NO_WAIT)
+    i = good.info
+    q, k, v = synth.make_qkv(T, H, W, G, d, 13, device="cuda", dtype=torch.bfloat16)
+    natural = bool(extra & tra.TRA_FLAG_NATURAL)
+    qi, ki, vi = (q, k, v) if natural else (gh.to_tile_major(x, i) for x in (q, k, v))
+    Ht = good.new_entropy() if natural else torch.empty(G, i.N_pad, device="cuda")
+    mask, out = good.new_mask(), good.new_out()
+    good.entropy(qi, ki, Ht)
+    good.radius_and_mask(Ht, mask)
+    torch.cuda.synchronize()
+    assert good.status() == 0
+    bad.attention(qi, ki, vi, mask, out)
+    torch.cuda.synchronize()
+    assert bad.status() == 5
+    bad.calibrate_topk(qi, ki, 0.9, 2)
+    torch.cuda.synchronize()
+    assert bad.status() == 5
+    good.attention(qi, ki, vi, mask, out)
+    Hc, Kc = good.calibrate_topk(qi, ki, 0.9, 2)
+    torch.cuda.synchronize()
+    assert good.status() == 0
+    o = out if natural else gh.to_natural(out, i)
+    assert torch.isfinite(o.float()).all()
+    assert int(Kc.max()) >= 1
+    good.close()
+    bad.close()
+
+
 @pytest.mark.parametrize("c", [CASES[1], CASES[4]], ids=_ids)
 def test_attention_bf16_output(c):
     """bf16 output: the fp32 result rounded once more; allowed error adds half a
