@@ -198,7 +198,7 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 # ---------------------------------------------------------------- oracle (CPU)
-def oracle_sample(wl, b, budget_s: float, rng_seed: int, heads=(0,), device="cuda"):
+def oracle_sample(wl, b, budget_s: float, rng_seed: int, heads=(0,), device="cuda", metric: int = 0):
     """Time the fp64 oracle's whole path (entropy, radius, attention) on a
     bounded random sample of queries of the same workload.  Returns the
     retained-pair TFLOP/s it reached and a description."""
@@ -225,10 +225,11 @@ def oracle_sample(wl, b, budget_s: float, rng_seed: int, heads=(0,), device="cud
         t0 = time.perf_counter()
         Hs = oracle.entropy(qb, kb, G, (T, H, W), d, key_stride=wl.key_stride, ktile=(8, 16), queries=idx) \
             if wl.key_stride == 1 else _oracle_entropy_tiled(oracle, qb, kb, G, wl, idx)
-        r, c, _ = oracle.radius(Hs.astype(np.float32), G, (T, H, W), wl.a, b, wl.gamma, wl.Rt, wl.Bmin, queries=idx)
+        r, c, _ = oracle.radius(Hs.astype(np.float32), G, (T, H, W), wl.a, b, wl.gamma, wl.Rt, wl.Bmin, queries=idx,
+                                metric=metric)
         r_all = np.zeros(G * N, np.int32)
         r_all[idx] = r
-        oracle.attention(qb, kb, vb, r_all, G, (T, H, W), d, wl.gamma, wl.Rt, queries=idx)
+        oracle.attention(qb, kb, vb, r_all, G, (T, H, W), d, wl.gamma, wl.Rt, queries=idx, metric=metric)
         dt = time.perf_counter() - t0
         return dt, int(c.sum()), nq
 
@@ -282,11 +283,14 @@ def oracle_parity(run, wl, n_queries: int = 256, seed: int = 77):
         Hr = oracle.entropy(qb, kb, 1, (T, H, W), d, queries=queries)
     else:
         Hr = _oracle_entropy_tiled(oracle, qb, kb, 1, wl, queries)
+    from sparse_attention_video_tra_b200 import TRA_FLAG_DISK
+    metric = oracle.DISK if run.plan.flags & TRA_FLAG_DISK else oracle.CHEBYSHEV
     rad = run.plan.mask_views(run.mask)[0][0].cpu().numpy()
-    r_ref, _, _ = oracle.radius(Hg, 1, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, queries=queries)
+    r_ref, _, _ = oracle.radius(Hg, 1, (T, H, W), wl.a, run.b, wl.gamma, wl.Rt, wl.Bmin, queries=queries,
+                                metric=metric)
     r_all = np.zeros(N, np.int32)
     r_all[nat[valid]] = rad[valid]
-    O = oracle.attention(qb, kb, vb, r_all, 1, (T, H, W), d, wl.gamma, wl.Rt, queries=queries)
+    O = oracle.attention(qb, kb, vb, r_all, 1, (T, H, W), d, wl.gamma, wl.Rt, queries=queries, metric=metric)
     Og = run.out[0].float().cpu().numpy()[rows]
     err = np.abs(Og - O)
     return {"queries": int(n_queries), "head": 0,
@@ -340,9 +344,9 @@ def attention_calls(args) -> int:
 def bench_config(args, wl, total_heads: int, world: int, b: float) -> dict:
     """The `config` object of the JSON line, the same for both arms: the
     workload, the batch, the plan's parameters and tile choice."""
-    from sparse_attention_video_tra_b200 import Plan
+    from sparse_attention_video_tra_b200 import Plan, TRA_FLAG_QSORT
     sharded = args.shard == "heads"
-    flags = query_group_flags(args.qsort, wl)
+    flags = plan_flags(args, wl)
     p = Plan(wl.T, wl.H, wl.W, 1, wl.d, wl.a, b, wl.gamma, wl.Rt, wl.Bmin, flags)
     tile_desc = f"1x{p.info.tile_h}x{p.info.tile_w}"
     p.close()
@@ -353,7 +357,8 @@ def bench_config(args, wl, total_heads: int, world: int, b: float) -> dict:
             "attention_calls_per_step": attention_calls(args),
             "a": wl.a, "b": round(float(b), 6), "gamma": wl.gamma, "Rt": wl.Rt, "Bmin": wl.Bmin,
             "tile": tile_desc,
-            "query_groups": "radius-sorted groups (TRA_FLAG_QSORT)" if flags else "spatial tiles",
+            "query_groups": "radius-sorted groups (TRA_FLAG_QSORT)" if flags & TRA_FLAG_QSORT else "spatial tiles",
+            "metric": "Euclidean disk (TRA_FLAG_DISK)" if args.metric == "disk" else "Chebyshev square",
             "inputs": "resident in HBM, larger than L2; L2 flushed before every step"}
 
 
@@ -370,11 +375,11 @@ def run_reference(args, rank, world):
     # target-fraction run finds its own, with the oracle on a query sample
     b = wl.b
     if b is None:
-        b = _oracle_calibrate_b(oracle, wl, dev)
+        b = _oracle_calibrate_b(oracle, wl, dev, oracle_metric(args))
     vals = []
     budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup + args.steps):
-        v, desc = oracle_sample(wl, b, budget, 1234 + s, device=dev)
+        v, desc = oracle_sample(wl, b, budget, 1234 + s, device=dev, metric=oracle_metric(args))
         if s >= args.warmup:
             vals.append((v, desc))
     value = float(np.mean([v for v, _ in vals]))
@@ -401,7 +406,7 @@ def synth_name(args, total_heads: int) -> str:
     return wl.name.replace(f"{wl.heads} heads", f"{total_heads} heads")
 
 
-def _oracle_calibrate_b(oracle, wl, dev):
+def _oracle_calibrate_b(oracle, wl, dev, metric: int = 0):
     from sparse_attention_video_tra_b200 import synth
     q, k, _ = synth.make_qkv(wl.T, wl.H, wl.W, wl.heads, wl.d, synth.SEED_BASE + wl.index, device=dev,
                              dtype=torch.bfloat16)
@@ -417,7 +422,8 @@ def _oracle_calibrate_b(oracle, wl, dev):
     lo, hi = -30.0, 30.0
     for _ in range(30):
         mid = 0.5 * (lo + hi)
-        _, c, _ = oracle.radius(Hs.astype(np.float32), 1, wl.grid, wl.a, mid, wl.gamma, wl.Rt, wl.Bmin, queries=idx)
+        _, c, _ = oracle.radius(Hs.astype(np.float32), 1, wl.grid, wl.a, mid, wl.gamma, wl.Rt, wl.Bmin, queries=idx,
+                                metric=metric)
         if c.mean() / wl.N < wl.target_retained:
             lo = mid
         else:
@@ -444,6 +450,18 @@ def query_group_flags(mode: str, wl) -> int:
     return TRA_FLAG_QSORT if (mode == "on" or rows > 1) else 0
 
 
+def plan_flags(args, wl) -> int:
+    """The plan flags of a run: query groups (above) and the spatial test."""
+    from sparse_attention_video_tra_b200 import TRA_FLAG_DISK
+    return query_group_flags(args.qsort, wl) | (TRA_FLAG_DISK if args.metric == "disk" else 0)
+
+
+def oracle_metric(args) -> int:
+    sys.path.insert(0, ROOT)
+    import oracle
+    return oracle.DISK if args.metric == "disk" else oracle.CHEBYSHEV
+
+
 def run_tra(args, rank, world):
     sys.path.insert(0, ROOT)
     from sparse_attention_video_tra_b200.runner import WorkloadRun
@@ -451,7 +469,7 @@ def run_tra(args, rank, world):
     wl, total_heads, _ = bench_workload(args, rank, world)
     args.workload_name = synth_name(args, total_heads)
     calls = attention_calls(args)
-    flags = query_group_flags(args.qsort, wl)
+    flags = plan_flags(args, wl)
     run = WorkloadRun(wl, calls=calls, seed_offset=rank, flags=flags)
     dev_idx = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
@@ -539,7 +557,7 @@ def run_tra(args, rank, world):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, desc = oracle_sample(wl, run.b, args.cpu_budget, 4321)
+        v, desc = oracle_sample(wl, run.b, args.cpu_budget, 4321, metric=oracle_metric(args))
         cpu = {"value": v, "unit": "TFLOP/s", "cores": desc["threads"], "kind": "oracle",
                "sample": f"{desc['queries']} random queries of head 0: entropy+radius+attention in fp64, "
                          f"{desc['seconds']} s",
@@ -707,6 +725,8 @@ def main(argv=None):
     ap.add_argument("--retained", type=float, default=0.0,
                     help="target retained fraction for calibrating b (0 = the workload's own)")
     ap.add_argument("--b", type=float, default=None, help="budget offset b (default: the workload's)")
+    ap.add_argument("--metric", default="square", choices=["square", "disk"],
+                    help="spatial test: the Chebyshev square (default) or the Euclidean disk (TRA_FLAG_DISK)")
     ap.add_argument("--qsort", default="auto", choices=["auto", "on", "off"],
                     help="radius-sorted query groups (TRA_FLAG_QSORT): auto = when the frame has an even "
                          "number of tile columns")
