@@ -68,13 +68,43 @@ __device__ __forceinline__ CountCtx count_ctx(const Geom& G, int t, int h, int w
     return x;
 }
 
+// The disk-row table of half-width s (s <= disk_smax): entry k <= s holds the
+// row half-width f_s(k) = isqrt(s^2 - k^2) (low 16 bits) and the running sum
+// F_s(k) = f_s(0) + ... + f_s(k) (high 16 bits; F_s(s) <= s (s + 1) < 2^16).
+// Row s starts at entry s (s + 1) / 2.
+__device__ __forceinline__ const uint32_t* disk_row(const uint32_t* dtab, int s)
+{
+    return dtab + (s * (s + 1) >> 1);
+}
+
+// sum over key rows k = 0 .. n (n <= s) of min(cap, f_s(k)): f_s decreases,
+// and f_s(k) >= cap  <=>  k^2 <= s^2 - cap^2  <=>  k <= f_s(cap) for cap < s,
+// so the rows up to J = f_s(cap) contribute cap each and the rest f_s(k)
+__device__ __forceinline__ int disk_capped_sum(const uint32_t* row, int s, int n, int cap)
+{
+    if (cap >= s) return (int)(row[n] >> 16);
+    const int J = (int)(row[cap] & 0xffffu);
+    return n <= J ? cap * (n + 1) : cap * (J + 1) + (int)(row[n] >> 16) - (int)(row[J] >> 16);
+}
+
 // in-frame clipped count at half-width s: the Chebyshev square is a clipped
 // rectangle; the disk sums, key row by key row, the clipped width
-// 2*isqrt(s^2 - dh^2) + 1
+// min(w, f) + min(W-1-w, f) + 1 with f = isqrt(s^2 - dh^2) -- from the
+// disk-row table in O(1) when there is one (s >= disk_smax covers the frame,
+// so s is capped there), else row by row
 template <bool DISK>
-__device__ __forceinline__ int frame_count(const Geom& G, const CountCtx& x, int s)
+__device__ __forceinline__ int frame_count(const Geom& G, const CountCtx& x, int s, const uint32_t* dtab)
 {
     if constexpr (DISK) {
+        if (dtab) {
+            const int sc = min(s, G.disk_smax);
+            const uint32_t* row = disk_row(dtab, sc);
+            const int up = min(sc, x.h), dn = min(sc, x.hb);
+            // rows h .. h - up and h .. h + dn; row h is in both
+            const int cu = up + 1 + disk_capped_sum(row, sc, up, x.w) + disk_capped_sum(row, sc, up, x.wb);
+            const int cd = dn + 1 + disk_capped_sum(row, sc, dn, x.w) + disk_capped_sum(row, sc, dn, x.wb);
+            return cu + cd - (min(x.w, sc) + min(x.wb, sc) + 1);
+        }
         // key rows h - k (k <= up) and h + k (k <= dn) share the half-width
         // isqrt(s^2 - k^2)
         const int sc = min(s, TRA_DISK_S_CLAMP);
@@ -94,12 +124,13 @@ __device__ __forceinline__ int frame_count(const Geom& G, const CountCtx& x, int
 
 // clipped neighbourhood count c(r) (at most N < 2^31)
 template <bool DISK>
-__device__ __forceinline__ long long nbr_count(const Geom& G, const uint16_t* tab, const CountCtx& x, int r)
+__device__ __forceinline__ long long nbr_count(const Geom& G, const uint16_t* tab, const uint32_t* dtab,
+                                               const CountCtx& x, int r)
 {
     int one = 0, two = 0;
-    for (int dl = 1; dl <= x.lo; ++dl) two += frame_count<DISK>(G, x, hw_at(G, tab, r, dl));
-    for (int dl = x.lo + 1; dl <= x.hi; ++dl) one += frame_count<DISK>(G, x, hw_at(G, tab, r, dl));
-    return (long long)frame_count<DISK>(G, x, hw_at(G, tab, r, 0)) + 2ll * two + one;
+    for (int dl = 1; dl <= x.lo; ++dl) two += frame_count<DISK>(G, x, hw_at(G, tab, r, dl), dtab);
+    for (int dl = x.lo + 1; dl <= x.hi; ++dl) one += frame_count<DISK>(G, x, hw_at(G, tab, r, dl), dtab);
+    return (long long)frame_count<DISK>(G, x, hw_at(G, tab, r, 0), dtab) + 2ll * two + one;
 }
 
 // Bhat = ceil(min(N, max(Bmin, exp(a*H + b)))): a*H and + b rounded
@@ -113,30 +144,31 @@ __device__ __forceinline__ long long budget_hat(const Geom& G, float Hent)
 // r = the smallest r in [0, r_cap] whose neighbourhood count reaches bh (the
 // count is monotone in r; r_cap when none does); c = that count.
 template <bool DISK>
-__device__ __forceinline__ int find_radius(const Geom& G, const uint16_t* tab, int t, int h, int w, long long bh,
-                                           long long& c)
+__device__ __forceinline__ int find_radius(const Geom& G, const uint16_t* tab, const uint32_t* dtab, int t, int h,
+                                           int w, long long bh, long long& c)
 {
     const CountCtx x = count_ctx(G, t, h, w);
     int lo = 0, hi = G.r_cap;
-    if constexpr (DISK) {
-        // the disk lies inside the square of the same half-width, so its
-        // radius is at least the square's; search [r_sq, 2 r_sq + 2] when
-        // that bracket reaches the budget, else the rest up to r_cap
+    if (DISK && !dtab) {
+        // row-by-row disk counts: the disk lies inside the square of the same
+        // half-width, so its radius is at least the square's; search
+        // [r_sq, 2 r_sq + 2] when that bracket reaches the budget, else the
+        // rest up to r_cap
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (nbr_count<false>(G, tab, x, mid) >= bh) hi = mid; else lo = mid + 1;
+            if (nbr_count<false>(G, tab, dtab, x, mid) >= bh) hi = mid; else lo = mid + 1;
         }
         const int r2 = min(G.r_cap, 2 * lo + 2);
-        if (nbr_count<true>(G, tab, x, r2) >= bh) hi = r2;
+        if (nbr_count<true>(G, tab, dtab, x, r2) >= bh) hi = r2;
         else { lo = min(r2 + 1, G.r_cap); hi = G.r_cap; }
     }
     long long c_hi = -1;                  // the count at hi, once evaluated
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        const long long cm = nbr_count<DISK>(G, tab, x, mid);
+        const long long cm = nbr_count<DISK>(G, tab, dtab, x, mid);
         if (cm >= bh) { hi = mid; c_hi = cm; } else lo = mid + 1;
     }
-    c = c_hi >= 0 ? c_hi : nbr_count<DISK>(G, tab, x, lo);
+    c = c_hi >= 0 ? c_hi : nbr_count<DISK>(G, tab, dtab, x, lo);
     return lo;
 }
 
@@ -145,16 +177,22 @@ constexpr int MASK_MAX_ROWS = 128 * TRA_MAX_STRIP_TILES;
 
 // Dynamic shared memory of the mask kernel, sized from the plan so that small
 // reaches keep many CTAs resident.  In order: the half-width table (uint16,
-// when the plan has one), and per group u < U the column interval [lo, hi]
-// and the disk's full-column bits of every (frame distance, tile row), the
-// length of every list row (frame, tile row).
+// when the plan has one), the disk-row table (uint32, when the plan has one),
+// and per group u < U the column interval [lo, hi] and the disk's full-column
+// bits of every (frame distance, tile row), the length of every list row
+// (frame, tile row).
 __host__ __device__ inline int mask_tab_bytes(int rte, int r_cap, bool tab)
 {
     return tab ? ((rte + 1) * (r_cap + 1) * 2 + 15) & ~15 : 0;
 }
-__host__ __device__ inline int mask_smem_bytes(int rte, int nTh, int r_cap, bool tab, int U)
+__host__ __device__ inline int mask_disk_bytes(int disk_smax)
 {
-    return mask_tab_bytes(rte, r_cap, tab) + U * (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
+    return disk_smax >= 0 ? ((disk_smax + 1) * (disk_smax + 2) / 2 * 4 + 15) & ~15 : 0;
+}
+__host__ __device__ inline int mask_smem_bytes(int rte, int nTh, int r_cap, bool tab, int disk_smax, int U)
+{
+    return mask_tab_bytes(rte, r_cap, tab) + mask_disk_bytes(disk_smax) +
+           U * (3 * (rte + 1) * nTh + (2 * rte + 1) * nTh) * 4;
 }
 
 // MAXT: the block size the instance is built for (128 * U); the register
@@ -167,7 +205,9 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 8 : (MAXT == 384 ? 3 : 2))
     const int U = QS ? G.nTh : 1;                                 // tiles (and groups) of this CTA
     const int RS = G.nTh;                                         // stride of one frame distance
     const uint16_t* tab = G.hw_tab ? reinterpret_cast<const uint16_t*>(mask_dyn) : nullptr;
-    int* grp_base = reinterpret_cast<int*>(mask_dyn + mask_tab_bytes(G.rte, G.r_cap, G.hw_tab != 0));
+    const int tab_bytes = mask_tab_bytes(G.rte, G.r_cap, G.hw_tab != 0);
+    const uint32_t* dtab = DISK && G.disk_smax >= 0 ? reinterpret_cast<const uint32_t*>(mask_dyn + tab_bytes) : nullptr;
+    int* grp_base = reinterpret_cast<int*>(mask_dyn + tab_bytes + (DISK ? mask_disk_bytes(G.disk_smax) : 0));
     const int GS = 3 * (G.rte + 1) * RS + (2 * G.rte + 1) * RS;   // ints per group
     constexpr int QR = QS ? MASK_MAX_ROWS : 1;
     __shared__ int s_key[QR];                  // QS: warp-sorted keys (radius + 1) << 10 | strip row
@@ -198,6 +238,19 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 8 : (MAXT == 384 ? 3 : 2))
             for (int rr = tid; rr <= G.r_cap; rr += blockDim.x)
                 wtab[dl * (G.r_cap + 1) + rr] = (uint16_t)halfwidth(rr, G.g[dl]);
     }
+    if (dtab) {
+        // one disk row per thread: half-widths and their running sum
+        uint32_t* wd = reinterpret_cast<uint32_t*>(mask_dyn + tab_bytes);
+        for (int sd = tid; sd <= G.disk_smax; sd += blockDim.x) {
+            uint32_t* row = wd + (sd * (sd + 1) >> 1);
+            int acc = 0;
+            for (int k = 0; k <= sd; ++k) {
+                const int f = isqrt_floor(sd * sd - k * k);
+                acc += f;
+                row[k] = (uint32_t)f | ((uint32_t)acc << 16);
+            }
+        }
+    }
     int* s_lo = grp_base + u * GS;                                // [rte + 1][nTh]
     int* s_hi = s_lo + (G.rte + 1) * RS;                          // [rte + 1][nTh]
     uint32_t* s_fullbits = reinterpret_cast<uint32_t*>(s_hi + (G.rte + 1) * RS);   // disk: full tile columns
@@ -219,7 +272,7 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 8 : (MAXT == 384 ? 3 : 2))
     bool valid = h < G.H && w < G.W;
     int r = -1;
     long long c = 0;
-    if (valid) r = find_radius<DISK>(G, tab, t, h, w, budget_hat(G, Hent[io_row(G, g, t, h, w, strip_tile(u) * 128 + i)]), c);
+    if (valid) r = find_radius<DISK>(G, tab, dtab, t, h, w, budget_hat(G, Hent[io_row(G, g, t, h, w, strip_tile(u) * 128 + i)]), c);
     reinterpret_cast<int32_t*>(mask + G.off_radius)[(size_t)g * G.N_pad + (size_t)strip_tile(u) * 128 + i] = r;
 
     if constexpr (QS) {

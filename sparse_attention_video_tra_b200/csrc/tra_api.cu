@@ -183,11 +183,16 @@ extern "C" tra_status tra_radius_and_mask(tra_plan plan, const float* Hent, void
 {
     if (!plan || !Hent || !mask || !aligned(Hent, 4) || !aligned(mask, 256)) return TRA_ERR_INVALID_ARG;
     if (mask_bytes < plan->mask_bytes) return TRA_ERR_WORKSPACE;
-    const tra::Geom& G = plan->geom;
+    tra::Geom G = plan->geom;
     // one CTA per tile-column strip (query groups) or per tile
     const int U = G.qsort ? G.nTh : 1;
     const dim3 grid(G.qsort ? G.T * G.nTw : G.nQ, G.G);
-    const int smem = tra::mask_smem_bytes(G.rte, G.nTh, G.r_cap, G.hw_tab != 0, U);
+    int smem = tra::mask_smem_bytes(G.rte, G.nTh, G.r_cap, G.hw_tab != 0, G.disk_smax, U);
+    if (G.disk_smax >= 0 && smem > kMaxSmem - 16 * 1024) {
+        // no room for the disk-row table: count the disk row by row
+        G.disk_smax = -1;
+        smem = tra::mask_smem_bytes(G.rte, G.nTh, G.r_cap, G.hw_tab != 0, G.disk_smax, U);
+    }
     if (smem > kMaxSmem - 16 * 1024) return TRA_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t* m = (uint8_t*)mask;

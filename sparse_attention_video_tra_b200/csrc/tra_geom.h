@@ -11,6 +11,7 @@
 #define TRA_MAX_HW 256                // largest H and W (half-widths kept as bytes)
 #define TRA_MAX_STRIP_TILES 4         // tile rows per frame with radius-sorted query groups
 #define TRA_MAX_HW_TAB 8192           // half-width table entries (Rt'+1)(r_cap+1) kept in shared memory
+#define TRA_MAX_DISK_TAB 12288        // disk row half-width / running-sum entries (S+1)(S+2)/2 kept in shared memory
 #define TRA_ERRBIT_TIMEOUT 1u
 #define TRA_ERRBIT_CHECK 2u
 
@@ -33,6 +34,8 @@ struct Geom {
     int disk;                        // spatial test dh^2 + dw^2 <= s^2 instead of the Chebyshev square
     int qsort;                       // radius-sorted query groups of tile-column strips
     int hw_tab;                      // the mask kernel tabulates s(r, |dt|) for r <= r_cap
+    int disk_smax;                   // disk: the mask kernel tabulates the disk rows of half-widths
+                                     // 0 .. disk_smax (the frame's cover radius); -1: no table
 };
 
 }  // namespace tra

@@ -120,6 +120,9 @@ extern "C" tra_status tra_plan_create(tra_plan* out, int T, int H, int W, int he
     }
     G.r_cap = (int)r;
     G.disk = disk ? 1 : 0;
+    // a disk of half-width >= need covers the frame, so the mask kernel's
+    // disk-row table needs the half-widths 0 .. need only
+    G.disk_smax = disk && (need + 1) * (need + 2) / 2 <= TRA_MAX_DISK_TAB ? (int)need : -1;
 
     G.a = a; G.b = b; G.Bmin = Bmin;
     G.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
