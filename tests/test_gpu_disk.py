@@ -35,6 +35,11 @@ CASES = [
     (4, 19, 21, 2, 64, 0.6, 3, 2, 8),
     (3, 9, 70, 1, 128, 0.9, 2, 3, 32),
     (2, 45, 80, 1, 128, 0.8, 1, 8, 16),
+    # the mask kernel's disk-row table covers half-widths up to the frame's cover
+    # radius when (S+1)(S+2)/2 <= 12288 entries: 3x155 frames (S = 155) use it,
+    # 3x156 frames (S = 156) count the disk row by row
+    (2, 3, 155, 1, 64, 0.8, 1, 4, 0),
+    (2, 3, 156, 1, 64, 0.8, 1, 4, 0),
 ]
 
 
