@@ -62,3 +62,31 @@ def test_query_group_default_follows_the_plan():
     assert bench.query_group_flags("auto", tall) == 0
     with pytest.raises(TraError):
         bench.query_group_flags("on", tall)
+
+
+def test_metric_switch_selects_the_disk_plans_and_oracle_metric():
+    """`--metric disk` adds TRA_FLAG_DISK to the plan flags and sends the
+    oracle legs to the oracle's disk metric; the default stays the Chebyshev
+    square.  The reference arm's line names the spatial test it ran."""
+    import argparse
+    import json
+    import subprocess
+    import sys
+    import oracle
+    from sparse_attention_video_tra_b200 import TRA_FLAG_DISK, synth
+    wl = synth.WORKLOADS["tiny"]
+    disk = argparse.Namespace(qsort="off", metric="disk")
+    square = argparse.Namespace(qsort="off", metric="square")
+    assert bench.plan_flags(disk, wl) == TRA_FLAG_DISK
+    assert bench.plan_flags(square, wl) == 0
+    assert bench.oracle_metric(disk) == oracle.DISK
+    assert bench.oracle_metric(square) == oracle.CHEBYSHEV
+    names = {}
+    for m in ("square", "disk"):
+        p = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--metric", m,
+                            "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+        assert p.returncode == 0, p.stderr[-3000:]
+        line = [json.loads(x) for x in p.stdout.splitlines() if x.startswith("{")][-1]
+        assert line["impl"] == "reference" and line["value"] > 0
+        names[m] = line["config"]["metric"]
+    assert names == {"square": "Chebyshev square", "disk": "Euclidean disk (TRA_FLAG_DISK)"}
