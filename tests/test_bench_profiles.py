@@ -1,7 +1,8 @@
-"""Host checks of the bench's roofline bookkeeping: the committed ncu traffic
-summary of the dominant kernel is found under the name the bench looks up,
-and its DRAM bytes are reported only while the kernel source it was taken on
-is unchanged."""
+"""Host checks of the bench's bookkeeping: the committed ncu traffic summary
+of the dominant kernel is found under the name the bench looks up, and its
+DRAM bytes are reported only while the kernel source it was taken on is
+unchanged; the --metric switch picks the plans' and the oracle's spatial
+test together."""
 import os
 
 import bench
