@@ -551,6 +551,11 @@ def run_tra(args, rank, world):
               "entropy_roofline": {"bound": "alu", "unit": "exponentials/s", "achieved": ent_rate,
                                    "peak": MUFU_EX2_PER_S, "frac": round(ent_rate / MUFU_EX2_PER_S, 4),
                                    "peak_derivation": "one ex2 per scored pair; MUFU 16/clk/SM x 148 SMs x 1965 MHz",
+                                   # the same bound at the median SM clock sampled over the
+                                   # timed region (entropy is about a sixth of it; the long
+                                   # kernels run at the power cap, below the 1965 MHz maximum)
+                                   "frac_at_sampled_clock": (round(ent_rate / (16 * 148 * clk["sm_mhz"] * 1e6), 4)
+                                                             if clk and clk.get("sm_mhz") else None),
                                    "dram_gbs": round(ent_bytes / ent_s / 1e9, 2),
                                    "dram_frac": round(ent_bytes / ent_s / 1e9 / hbm, 5),
                                    "algorithmic_bytes": ent_bytes}}
