@@ -11,7 +11,8 @@ the mask slot of the strip's tile in tile row u.  Checked here:
   members' counts;
 * attention within max-abs 1e-2 / mean-abs 1e-3 of the fp64 oracle, with the
   Chebyshev square and the disk;
-* the natural layout gives the tile-major results bit for bit.
+* the natural layout gives the tile-major results bit for bit;
+* bf16 output (TRA_FLAG_OUT_BF16) equals the fp32 output rounded to bf16.
 
 Definitions: "Token Radius Attention for Efficient Video Generation"
 (gist.science summary), section 2; the grouping is a scheduling choice of
@@ -152,3 +153,45 @@ def test_natural_layout_is_bit_identical():
         assert torch.equal(a, b)
     assert torch.equal(tm.group_view(m_tm), nat.group_view(m_n))
     assert torch.equal(gh.to_natural(o_tm, i), o_n)
+
+
+@pytest.mark.parametrize("natural", [False, True], ids=["tile-major", "natural"])
+@pytest.mark.parametrize("metric", [oracle.CHEBYSHEV, oracle.DISK], ids=["square", "disk"])
+@pytest.mark.parametrize("c", [CASES[1], CASES[4], CASES[6]], ids=_ids)
+def test_bf16_output_is_the_rounded_fp32_output(c, metric, natural):
+    """With query groups each softmax thread writes its own query's row through
+    the group map; the bf16 epilogue (TRA_FLAG_OUT_BF16) rounds the same fp32
+    value the fp32 epilogue stores, so its rows equal the fp32 rows rounded to
+    bf16 (round to nearest even), bit for bit, at every query."""
+    T, H, W, G, d, gamma, Rt, Bmin, _ = c
+    N = T * H * W
+    rng = np.random.default_rng(29 + sum(c[:5]))
+    flags = tra.TRA_FLAG_QSORT | (tra.TRA_FLAG_DISK if metric == oracle.DISK else 0) | \
+        (tra.TRA_FLAG_NATURAL if natural else 0)
+    p32 = _plan(c, 1.0, math.log(0.4), flags)
+    p16 = _plan(c, 1.0, math.log(0.4), flags | tra.TRA_FLAG_OUT_BF16)
+    i = p32.info
+    q, k, v = synth.make_qkv(T, H, W, G, d, 37 + sum(c[:5]), device="cuda", dtype=torch.bfloat16)
+    Hn = torch.from_numpy(rng.uniform(0.0, math.log(N), size=(G, N)).astype(np.float32)).cuda()
+    if natural:
+        qi, ki, vi, Hi = q, k, v, Hn
+    else:
+        qi, ki, vi = (gh.to_tile_major(x, i) for x in (q, k, v))
+        Hi = gh.to_tile_major(Hn, i)
+    m32, m16 = p32.new_mask(), p16.new_mask()
+    p32.radius_and_mask(Hi, m32)
+    p16.radius_and_mask(Hi, m16)
+    o32, o16 = p32.new_out(), p16.new_out()
+    assert o32.dtype == torch.float32 and o16.dtype == torch.bfloat16
+    p32.attention(qi, ki, vi, m32, o32)
+    p16.attention(qi, ki, vi, m16, o16)
+    torch.cuda.synchronize()
+    assert p32.status() == 0 and p16.status() == 0
+    for a, b in zip(p32.mask_views(m32)[:3], p16.mask_views(m16)[:3]):
+        assert torch.equal(a, b)
+    assert torch.equal(p32.group_view(m32), p16.group_view(m16))
+    if not natural:
+        o32, o16 = gh.to_natural(o32, i), gh.to_natural(o16, i)
+    assert torch.equal(o16.view(torch.int16), o32.to(torch.bfloat16).view(torch.int16))
+    p32.close()
+    p16.close()
