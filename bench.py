@@ -49,6 +49,17 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def peak_value(key: str):
+    """One roofline denominator: (value, "measured"|"fallback").  The measured
+    file's number when it holds one under `key`, else the profiling recipe's
+    fallback, labelled as such."""
+    pk, kind = peaks()
+    v = pk.get(key) if isinstance(pk, dict) else None
+    if kind == "measured" and isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+        return float(v), "measured"
+    return float(FALLBACK_PEAKS[key]), "fallback"
+
+
 # ---------------------------------------------------------------- distributed
 def dist_setup(expected_world: int = 0):
     """Rank and world size from the torchrun environment; one process per GPU
@@ -523,10 +534,9 @@ def run_tra(args, rank, world):
         mask_runs.append(a0.elapsed_time(a1))
     mask_cold_ms = float(np.median(mask_runs))
 
-    pk, pk_kind = peaks()
     avg_call_s = float(np.median(call_ms)) / 1000.0
     achieved = flops / avg_call_s / 1e12
-    peak = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak, pk_kind = peak_value("bf16_tflops_sustained")
     computed = run.computed_pairs()
     traffic = recorded_traffic(ROOFLINE_KERNEL, args.workload)
     roofline = {"bound": "tensor", "kernel": "tra::" + ROOFLINE_KERNEL, "achieved": round(achieved, 2),
@@ -535,9 +545,9 @@ def run_tra(args, rank, world):
                 "computed_tile_tflops": round(4.0 * wl.d * computed / avg_call_s / 1e12, 2),
                 "computed_tile_frac": round(4.0 * wl.d * computed / avg_call_s / 1e12 / peak, 4),
                 "tile_efficiency": round(run.retained_pairs / computed, 4),
-                "frac_of_burst": round(achieved / float(pk.get("bf16_tflops", 1590.0)), 4)}
+                "frac_of_burst": round(achieved / peak_value("bf16_tflops")[0], 4)}
     mask_bytes_alg = mask_algorithmic_bytes(run)
-    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    hbm, hbm_kind = peak_value("hbm_gbs")
     ent_s = float(np.median(ent_ms)) / 1000.0
     ent_rate = run.entropy_pairs() / ent_s
     ent_bytes = entropy_algorithmic_bytes(run)
@@ -546,6 +556,7 @@ def run_tra(args, rank, world):
               "mask_ms_l2_flushed": round(mask_cold_ms, 4),
               "mask_gbs": round(mask_bytes_alg / (mask_cold_ms / 1000.0) / 1e9, 2),
               "mask_hbm_frac": round(mask_bytes_alg / (mask_cold_ms / 1000.0) / 1e9 / hbm, 4),
+              "hbm_peak": {"gbs": hbm, "kind": hbm_kind},
               "attention_ms_per_call": round(avg_call_s * 1000.0, 3),
               "entropy_scores_per_s": ent_rate,
               "entropy_roofline": {"bound": "alu", "unit": "exponentials/s", "achieved": ent_rate,

@@ -91,3 +91,15 @@ def test_metric_switch_selects_the_disk_plans_and_oracle_metric():
         assert line["impl"] == "reference" and line["value"] > 0
         names[m] = line["config"]["metric"]
     assert names == {"square": "Chebyshev square", "disk": "Euclidean disk (TRA_FLAG_DISK)"}
+
+
+def test_peaks_are_labelled_by_their_source(tmp_path, monkeypatch):
+    """Each roofline denominator is the measured file's number when the file
+    holds one under that key, else the recipe's fallback, labelled as such."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.peak_value("bf16_tflops_sustained") == (1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6537.0, "bf16_tflops": "n/a"}))
+    assert bench.peak_value("hbm_gbs") == (6537.0, "measured")
+    assert bench.peak_value("bf16_tflops") == (1590.0, "fallback")
+    assert bench.peak_value("bf16_tflops_sustained") == (1400.0, "fallback")
