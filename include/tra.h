@@ -128,7 +128,8 @@ typedef struct {
     int n_tiles_h, n_tiles_w;
     int n_tiles;           /* tiles per head = T * n_tiles_h * n_tiles_w */
     int rt_eff;            /* Rt' = min(Rt, T-1) */
-    int r_cap;             /* smallest r with floor(r*gamma^Rt' + 1e-9) >= max(H,W)-1 */
+    int r_cap;             /* smallest r with s = floor(r*gamma^Rt' + 1e-9) >= max(H,W)-1;
+                              with TRA_FLAG_DISK, s^2 >= (H-1)^2 + (W-1)^2 */
     int list_cap;          /* max key tiles listed per query tile = (2Rt'+1) * tiles/frame */
     size_t mask_bytes;     /* size of the mask buffer tra_radius_and_mask fills */
     /* byte offsets inside the mask buffer (each 256-byte aligned):
