@@ -216,28 +216,24 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     __syncthreads();
     {
+        // one thread per bit position: an entry's rank in its class is its
+        // word's class offset plus the class bits below it in the word
         const int nAo = s_cls[0], nBo = s_cls[1], m2 = min(nAo, nBo);
-        for (int w = tid; w < L.bw; w += C::THREADS) {
-            const uint32_t ia = bits[w], ib = bits[L.bw + w], fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
-#pragma unroll
-            for (int c = 0; c < 3; ++c) {
-                uint32_t m = c == 0 ? (ia & ~ib) : (c == 1 ? (ib & ~ia) : (ia & ib));
-                int k = (int)bits[(4 + c) * L.bw + w];      // rank of the word's first entry in its class
-                while (m) {
-                    const int b = __ffs(m) - 1;
-                    m &= m - 1;
-                    // A-only rank k goes to 2k, B-only to 2k + 1 while both
-                    // classes last; the longer one's rest follows; then both
-                    const int pos = c == 2 ? nAo + nBo + k : (k < m2 ? 2 * k + c : m2 + k);
-                    ++k;
-                    int tk, trk, tck;
-                    tile_coords(G, base + 32 * w + b, tk, trk, tck);
-                    const uint32_t bit = 1u << b;
-                    merged[pos] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) |
-                                  ((ib & bit) ? (MT_IN0 << 1) : 0u) | ((fa & bit) ? MT_FULL0 : 0u) |
-                                  ((fb & bit) ? (MT_FULL0 << 1) : 0u);
-                }
-            }
+        for (int idx = tid; idx < 32 * L.bw; idx += C::THREADS) {
+            const int w = idx >> 5, b = idx & 31;
+            const uint32_t ia = bits[w], ib = bits[L.bw + w], bit = 1u << b;
+            if (!((ia | ib) & bit)) continue;
+            const int c = (ia & bit) ? ((ib & bit) ? 2 : 0) : 1;
+            const uint32_t m = c == 0 ? (ia & ~ib) : (c == 1 ? (ib & ~ia) : (ia & ib));
+            const int k = (int)bits[(4 + c) * L.bw + w] + __popc(m & (bit - 1u));
+            // A-only rank k goes to 2k, B-only to 2k + 1 while both classes
+            // last; the longer one's rest follows; then the tiles both list
+            const int pos = c == 2 ? nAo + nBo + k : (k < m2 ? 2 * k + c : m2 + k);
+            const uint32_t fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
+            int tk, trk, tck;
+            tile_coords(G, base + idx, tk, trk, tck);
+            merged[pos] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) | ((ib & bit) ? (MT_IN0 << 1) : 0u) |
+                          ((fa & bit) ? MT_FULL0 : 0u) | ((fb & bit) ? (MT_FULL0 << 1) : 0u);
         }
     }
     if (tid == 0) {
