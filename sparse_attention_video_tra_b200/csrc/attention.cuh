@@ -268,20 +268,36 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         int tqa_, tra_, tca_, tqb_, trb_, tcb_;
         tile_coords(G, qa, tqa_, tra_, tca_);
         tile_coords(G, hasB ? qb : qa, tqb_, trb_, tcb_);
-        for (int e = tid; e < 128 * np * CH; e += C::THREADS) {
-            const int d = e / CH, ch = e - d * CH;
-            const int sl = d >> 7, dr = d & 127;
-            const int l = (sl ? grp_b : grp_a)[dr];
-            const int tq = sl ? tqb_ : tqa_, tcq = sl ? tcb_ : tca_;
-            const int hq = (l >> 7) * G.th + ((l & 127) >> TWL), wq = tcq * TW + (l & (TW - 1));
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (hq < G.H && wq < G.W) {
-                const int tl = (tq * G.nTh + (l >> 7)) * G.nTw + tcq;
-                const size_t qrow = io_row(G, g, tq, hq, wq, tl * 128 + (l & 127));
-                val = __ldg(reinterpret_cast<const uint4*>(qraw) + qrow * CH + ch);
+        // batches of QB independent loads (all in flight at once), then their stores
+        constexpr int QB = 4;
+        for (int e0 = tid; e0 < 128 * np * CH; e0 += QB * C::THREADS) {
+            uint4 qv[QB];
+#pragma unroll
+            for (int k = 0; k < QB; ++k) {
+                const int e = e0 + k * C::THREADS;
+                qv[k] = make_uint4(0u, 0u, 0u, 0u);
+                if (e < 128 * np * CH) {
+                    const int d = e / CH, ch = e - d * CH;
+                    const int sl = d >> 7, dr = d & 127;
+                    const int l = (sl ? grp_b : grp_a)[dr];
+                    const int tq = sl ? tqb_ : tqa_, tcq = sl ? tcb_ : tca_;
+                    const int hq = (l >> 7) * G.th + ((l & 127) >> TWL), wq = tcq * TW + (l & (TW - 1));
+                    if (hq < G.H && wq < G.W) {
+                        const int tl = (tq * G.nTh + (l >> 7)) * G.nTw + tcq;
+                        const size_t qrow = io_row(G, g, tq, hq, wq, tl * 128 + (l & 127));
+                        qv[k] = __ldg(reinterpret_cast<const uint4*>(qraw) + qrow * CH + ch);
+                    }
+                }
             }
-            const int pn = ch >> 3, cc = ch & 7;
-            *reinterpret_cast<uint4*>(sQ + sl * C::TILE + pn * C::PANEL + dr * 128 + ((cc ^ (dr & 7)) << 4)) = val;
+#pragma unroll
+            for (int k = 0; k < QB; ++k) {
+                const int e = e0 + k * C::THREADS;
+                if (e < 128 * np * CH) {
+                    const int d = e / CH, ch = e - d * CH;
+                    const int sl = d >> 7, dr = d & 127, pn = ch >> 3, cc = ch & 7;
+                    *reinterpret_cast<uint4*>(sQ + sl * C::TILE + pn * C::PANEL + dr * 128 + ((cc ^ (dr & 7)) << 4)) = qv[k];
+                }
+            }
         }
         fence_proxy_async_smem();                               // generic smem writes -> tensor-core reads
         __syncthreads();
