@@ -190,50 +190,90 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (e & 0x8000) atomicOr(&bits[(isB ? 3 : 2) * L.bw + (bit >> 5)], 1u << (bit & 31));
     }
     __syncthreads();
-    if (warp == 0) {
-        int carry[3] = {0, 0, 0};
-        for (int w0 = 0; w0 < L.bw; w0 += 32) {
-            const int w = w0 + lane;
-            const uint32_t ia = w < L.bw ? bits[w] : 0u, ib = w < L.bw ? bits[L.bw + w] : 0u;
-            const uint32_t cls[3] = {ia & ~ib, ib & ~ia, ia & ib};
+    if (L.bw <= 32) {
+        // every warp scans the (at most 32) words itself, in registers: lane j
+        // holds word j's class counts and their exclusive prefix, so no
+        // barrier is needed before the expansion
+        const uint32_t ja = lane < L.bw ? bits[lane] : 0u, jb = lane < L.bw ? bits[L.bw + lane] : 0u;
+        int ex[3], tot[3];
 #pragma unroll
-            for (int c = 0; c < 3; ++c) {
-                const int cnt = __popc(cls[c]);
-                int incl = cnt;
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                if (w < L.bw) bits[(4 + c) * L.bw + w] = carry[c] + incl - cnt;
-                carry[c] += __shfl_sync(0xffffffffu, incl, 31);
+        for (int c = 0; c < 3; ++c) {
+            const int cnt = __popc(c == 0 ? (ja & ~jb) : (c == 1 ? (jb & ~ja) : (ja & jb)));
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
             }
+            ex[c] = incl - cnt;
+            tot[c] = __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) {
-            s_cls[0] = carry[0];
-            s_cls[1] = carry[1];
-            *s_n = carry[0] + carry[1] + carry[2];
-        }
-    }
-    __syncthreads();
-    {
-        // one thread per bit position: an entry's rank in its class is its
-        // word's class offset plus the class bits below it in the word
-        const int nAo = s_cls[0], nBo = s_cls[1], m2 = min(nAo, nBo);
+        if (tid == 0) *s_n = tot[0] + tot[1] + tot[2];
+        const int nAo = tot[0], nBo = tot[1], m2 = min(nAo, nBo);
+        // one thread per bit position; a warp's 32 positions are one word, so
+        // the word's class offsets come from its lane by shuffle
         for (int idx = tid; idx < 32 * L.bw; idx += C::THREADS) {
             const int w = idx >> 5, b = idx & 31;
+            const int o0 = __shfl_sync(0xffffffffu, ex[0], w), o1 = __shfl_sync(0xffffffffu, ex[1], w),
+                      o2 = __shfl_sync(0xffffffffu, ex[2], w);
             const uint32_t ia = bits[w], ib = bits[L.bw + w], bit = 1u << b;
             if (!((ia | ib) & bit)) continue;
             const int c = (ia & bit) ? ((ib & bit) ? 2 : 0) : 1;
             const uint32_t m = c == 0 ? (ia & ~ib) : (c == 1 ? (ib & ~ia) : (ia & ib));
-            const int k = (int)bits[(4 + c) * L.bw + w] + __popc(m & (bit - 1u));
-            // A-only rank k goes to 2k, B-only to 2k + 1 while both classes
-            // last; the longer one's rest follows; then the tiles both list
+            const int k = (c == 0 ? o0 : (c == 1 ? o1 : o2)) + __popc(m & (bit - 1u));
             const int pos = c == 2 ? nAo + nBo + k : (k < m2 ? 2 * k + c : m2 + k);
             const uint32_t fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
             int tk, trk, tck;
             tile_coords(G, base + idx, tk, trk, tck);
             merged[pos] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) | ((ib & bit) ? (MT_IN0 << 1) : 0u) |
                           ((fa & bit) ? MT_FULL0 : 0u) | ((fb & bit) ? (MT_FULL0 << 1) : 0u);
+        }
+    } else {
+        if (warp == 0) {
+            int carry[3] = {0, 0, 0};
+            for (int w0 = 0; w0 < L.bw; w0 += 32) {
+                const int w = w0 + lane;
+                const uint32_t ia = w < L.bw ? bits[w] : 0u, ib = w < L.bw ? bits[L.bw + w] : 0u;
+                const uint32_t cls[3] = {ia & ~ib, ib & ~ia, ia & ib};
+#pragma unroll
+                for (int c = 0; c < 3; ++c) {
+                    const int cnt = __popc(cls[c]);
+                    int incl = cnt;
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    if (w < L.bw) bits[(4 + c) * L.bw + w] = carry[c] + incl - cnt;
+                    carry[c] += __shfl_sync(0xffffffffu, incl, 31);
+                }
+            }
+            if (lane == 0) {
+                s_cls[0] = carry[0];
+                s_cls[1] = carry[1];
+                *s_n = carry[0] + carry[1] + carry[2];
+            }
+        }
+        __syncthreads();
+        {
+            // one thread per bit position: an entry's rank in its class is its
+            // word's class offset plus the class bits below it in the word
+            const int nAo = s_cls[0], nBo = s_cls[1], m2 = min(nAo, nBo);
+            for (int idx = tid; idx < 32 * L.bw; idx += C::THREADS) {
+                const int w = idx >> 5, b = idx & 31;
+                const uint32_t ia = bits[w], ib = bits[L.bw + w], bit = 1u << b;
+                if (!((ia | ib) & bit)) continue;
+                const int c = (ia & bit) ? ((ib & bit) ? 2 : 0) : 1;
+                const uint32_t m = c == 0 ? (ia & ~ib) : (c == 1 ? (ib & ~ia) : (ia & ib));
+                const int k = (int)bits[(4 + c) * L.bw + w] + __popc(m & (bit - 1u));
+                // A-only rank k goes to 2k, B-only to 2k + 1 while both classes
+                // last; the longer one's rest follows; then the tiles both list
+                const int pos = c == 2 ? nAo + nBo + k : (k < m2 ? 2 * k + c : m2 + k);
+                const uint32_t fa = bits[2 * L.bw + w], fb = bits[3 * L.bw + w];
+                int tk, trk, tck;
+                tile_coords(G, base + idx, tk, trk, tck);
+                merged[pos] = pack_tile(tk, trk, tck) | ((ia & bit) ? MT_IN0 : 0u) | ((ib & bit) ? (MT_IN0 << 1) : 0u) |
+                              ((fa & bit) ? MT_FULL0 : 0u) | ((fb & bit) ? (MT_FULL0 << 1) : 0u);
+            }
         }
     }
     if (tid == 0) {
@@ -256,6 +296,22 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t* sK = smem + C::OFF_K;
     uint8_t* sV = smem + C::OFF_V;
     const int kbase = g * G.N_pad;
+    // the first ring-depth of K and V tiles goes out now, so that their
+    // latency overlaps the query gather
+    static_assert(C::KST == C::VST, "one ring depth for K and V");
+    const int pre = min(n, C::KST);
+    if ((warp == C::WARP_LOAD || warp == C::WARP_VLOAD) && lane == 0) {
+        const bool isK = warp == C::WARP_LOAD;
+        for (int j = 0; j < pre; ++j) {
+            const uint32_t e = merged[j];
+            const int tk = (int)(e & 0x7fff), trk = (int)((e >> 15) & 63), tck = (int)((e >> 21) & 31);
+            mbar_arrive_expect_tx(&(isK ? k_full : v_full)[j], C::TILE);
+#pragma unroll
+            for (int p = 0; p < C::NP; ++p)
+                load_tile_panel((isK ? sK : sV) + j * C::TILE + p * C::PANEL, isK ? &tm_k : &tm_v, G, p, g, tk, trk, tck,
+                                &(isK ? k_full : v_full)[j]);
+        }
+    }
     // radius-sorted query groups: row r of slot s holds strip row grp_s[r] of
     // the slot's strip (tile row grp >> 7, row grp & 127 of that tile)
     const uint16_t* grp_a = reinterpret_cast<const uint16_t*>(mask + G.off_group) + ((size_t)g * G.nQ + qa) * 128;
@@ -332,8 +388,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             uint64_t* emptyb = isK ? k_empty : v_empty;
             uint8_t* ring = isK ? sK : sV;
             const CUtensorMap* tm = isK ? &tm_k : &tm_v;
-            int iss = 0;
-            for (int j = 0; j < n; ++j) {
+            int iss = pre;                              // the first ring-depth went out before the gather
+            for (int j = pre; j < n; ++j) {
                 const uint32_t e = merged[j];
                 const int tk = (int)(e & 0x7fff), trk = (int)((e >> 15) & 63), tck = (int)((e >> 21) & 31);
                 const int st = j % ST;
